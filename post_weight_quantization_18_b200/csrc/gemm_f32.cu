@@ -1,0 +1,116 @@
+// gemm_f32.cu — C = alpha * op(A) op(B) + beta * C in fp32 (row-major), CUDA-core version.
+//
+// Serves the fp32 pieces of the path: the lazy trailing update W[:, F] -= Err_B U[B, F]
+// ("GPTQ: Mathematical Foundations ...", §2 Lazy Batch Updates), the GEMM steps of the
+// Cholesky / triangular-inverse recursion, and the Hessian of fp32 calibration inputs.
+// 128x128 output tile per 256-thread CTA, 8x8 outputs per thread, k-slabs of 16 staged in
+// shared memory (transposes resolved while staging).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace {
+
+constexpr int TM = 128, TN = 128, TK = 16, THREADS = 256;
+
+__global__ void __launch_bounds__(THREADS)
+gemm_f32_simt_kernel(int M, int N, int K, float alpha, const float* __restrict__ A, long long lda,
+                     int transA, const float* __restrict__ B, long long ldb, int transB,
+                     float beta, float* __restrict__ C, long long ldc, int upper_only,
+                     const int32_t* status) {
+  __shared__ __align__(16) float As[2][TK][TM + 4];
+  __shared__ __align__(16) float Bs[2][TK][TN + 4];
+  if (gptq::status_bad(status)) return;
+  const int m0 = blockIdx.y * TM, n0 = blockIdx.x * TN;
+  if (upper_only && m0 > n0 + TN - 1) return;  // tile entirely below the diagonal
+  const int tid = threadIdx.x;
+  const int tx = tid & 15, ty = tid >> 4;
+
+  auto load = [&](int buf, int k0) {
+    // A slab: op(A)[m0 + mm][k0 + kk], 128 x 16 = 2048 values, 8 per thread.
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int e = tid + r * THREADS;
+      int mm, kk;
+      if (transA) { mm = e & (TM - 1); kk = e >> 7; }   // consecutive threads along m
+      else { kk = e & (TK - 1); mm = e >> 4; }          // consecutive threads along k
+      const int gm = m0 + mm, gk = k0 + kk;
+      float v = 0.f;
+      if (gm < M && gk < K) v = transA ? A[(long long)gk * lda + gm] : A[(long long)gm * lda + gk];
+      As[buf][kk][mm] = v;
+    }
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int e = tid + r * THREADS;
+      int nn, kk;
+      if (!transB) { nn = e & (TN - 1); kk = e >> 7; }
+      else { kk = e & (TK - 1); nn = e >> 4; }
+      const int gn = n0 + nn, gk = k0 + kk;
+      float v = 0.f;
+      if (gn < N && gk < K) v = transB ? B[(long long)gn * ldb + gk] : B[(long long)gk * ldb + gn];
+      Bs[buf][kk][nn] = v;
+    }
+  };
+
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+
+  const int nk = (K + TK - 1) / TK;
+  if (nk > 0) load(0, 0);
+  __syncthreads();
+  for (int kt = 0; kt < nk; ++kt) {
+    const int cur = kt & 1;
+    if (kt + 1 < nk) load(cur ^ 1, (kt + 1) * TK);
+#pragma unroll
+    for (int kk = 0; kk < TK; ++kk) {
+      float a[8], b[8];
+      const float4 a0 = *reinterpret_cast<const float4*>(&As[cur][kk][ty * 4]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&As[cur][kk][64 + ty * 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[cur][kk][tx * 4]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[cur][kk][64 + tx * 4]);
+      a[0] = a0.x; a[1] = a0.y; a[2] = a0.z; a[3] = a0.w;
+      a[4] = a1.x; a[5] = a1.y; a[6] = a1.z; a[7] = a1.w;
+      b[0] = b0.x; b[1] = b0.y; b[2] = b0.z; b[3] = b0.w;
+      b[4] = b1.x; b[5] = b1.y; b[6] = b1.z; b[7] = b1.w;
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int gm = m0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + (i - 4));
+    if (gm >= M) continue;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int gn = n0 + (j < 4 ? tx * 4 + j : 64 + tx * 4 + (j - 4));
+      if (gn >= N) continue;
+      if (upper_only && gm > gn) continue;
+      float* cp = C + (long long)gm * ldc + gn;
+      const float v = alpha * acc[i][j];
+      *cp = (beta == 0.f) ? v : fmaf(beta, *cp, v);
+    }
+  }
+}
+
+}  // namespace
+
+namespace gptq_host {
+
+int gemm_f32(int M, int N, int K, float alpha, const float* A, long long lda, bool transA,
+             const float* B, long long ldb, bool transB, float beta, float* C, long long ldc,
+             bool upper_only, const int32_t* status, cudaStream_t stream) {
+  if (M <= 0 || N <= 0) return 0;
+  dim3 grid((N + TN - 1) / TN, (M + TM - 1) / TM);
+  gemm_f32_simt_kernel<<<grid, THREADS, 0, stream>>>(M, N, K, alpha, A, lda, transA ? 1 : 0, B,
+                                                     ldb, transB ? 1 : 0, beta, C, ldc,
+                                                     upper_only ? 1 : 0, status);
+  return cudaGetLastError() == cudaSuccess ? 0 : GPTQ_ERR_CUDA;
+}
+
+}  // namespace gptq_host

@@ -1,0 +1,51 @@
+// kernels.h — host-side launchers of the library's kernels (internal; not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gptq_host {
+
+// ---- Hessian ----
+int syrk_bf16_upper(float* H, int d, long long ldh, const void* X, long long n_tokens,
+                    long long ldx, float alpha, int accumulate, int32_t* status,
+                    cudaStream_t stream);
+
+// ---- fp32 GEMM: C = alpha * op(A) op(B) + beta * C, row-major; op(A) is M x K, op(B) K x N.
+// upper_only: only elements with row <= col of C are written (the rest is left untouched).
+int gemm_f32(int M, int N, int K, float alpha, const float* A, long long lda, bool transA,
+             const float* B, long long ldb, bool transB, float beta, float* C, long long ldc,
+             bool upper_only, const int32_t* status, cudaStream_t stream);
+
+// ---- prepare ----
+int prep_permute_sym(const float* H, float* Hp, const int32_t* perm, int d, cudaStream_t stream);
+int prep_copy_upper(const float* src, float* dst, int d, cudaStream_t stream);
+int prep_act_order(const float* H, int32_t* perm, int d, cudaStream_t stream);
+int prep_identity_perm(int32_t* perm, int d, cudaStream_t stream);
+int prep_dead_damp(float* H, uint8_t* dead, int d, float percdamp, int32_t* status,
+                   cudaStream_t stream);
+int prep_zero_lower(float* U, int d, cudaStream_t stream);
+int prep_base_block(float* Hblk, float* Ublk, int n, int ld, int index0, int32_t* status,
+                    cudaStream_t stream);
+constexpr int kPrepBase = 128;
+
+// ---- sweep ----
+int sweep_gather_w(const void* W, int w_dtype, long long ldw, int n, int d, const int32_t* perm,
+                   const uint8_t* dead, float* Wwork, const int32_t* status, cudaStream_t stream);
+int sweep_row_params(const float* Wwork, int n, int d, int bits, int sym, float* scales,
+                     float* zeros, const int32_t* status, cudaStream_t stream);
+int sweep_block(float* Wwork, const float* U, float* Err, uint8_t* codes, float* scales,
+                float* zeros, int n, int d, int col0, int bits, int group_size, int sym,
+                int32_t* status, cudaStream_t stream);
+int sweep_unpermute_codes(const uint8_t* codes_sweep, const int32_t* perm, uint8_t* codes, int n,
+                          int d, const int32_t* status, cudaStream_t stream);
+int sweep_g_idx(const int32_t* perm, int32_t* g_idx, int d, int group_size, cudaStream_t stream);
+
+// ---- RTN and pack ----
+int rtn_launch(const void* W, int w_dtype, long long ldw, int n, int d, int bits, int group_size,
+               int sym, uint8_t* codes, float* scales, float* zeros, cudaStream_t stream);
+int pack_launch(const uint8_t* codes, int n, int d, int bits, const float* scales,
+                const float* zeros, long long n_groups, uint32_t* qweight, uint16_t* scales_f16,
+                uint16_t* zeros_f16, cudaStream_t stream);
+
+}  // namespace gptq_host

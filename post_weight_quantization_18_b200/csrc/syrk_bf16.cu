@@ -1,0 +1,305 @@
+// syrk_bf16.cu — H_upper += alpha * X^T X for token-major bf16 X on tcgen05 tensor cores.
+//
+// Computes the layer Hessian H = 2 X X^T ("INT4 and GPTQ Quantization", §The Quantization Error
+// and Layerwise Objective; "GPTQ: Mathematical Foundations ...", §Second-Order Taylor Expansion
+// and the Hessian). X is stored token-major [N, d] (row t = one calibration token), so both
+// GEMM operands are X itself read "MN-major": element (t, i) sits at t*ldx + i.
+//
+// Design (one CTA per SM, persistent):
+//   * Work unit = (128 x 256 output tile with i-block <= j-block, token chunk). Only tiles that
+//     touch the upper triangle are scheduled; token chunks (split-K) are used only when the
+//     tiles alone cannot fill the SMs. Units are chunk-major so concurrently running CTAs
+//     share one L2-resident chunk of X.
+//   * warp 0: TMA producer — per 64-token k-block, two 64x64 boxes of X for the A tile (rows
+//     i0..i0+127) and four for the B tile (j0..j0+255), 128-byte swizzled, 4-stage ring.
+//   * warp 1: TMEM owner and MMA issuer — tcgen05.mma kind::f16, M=128, N=256, K=16, both
+//     operands MN-major; fp32 accumulators double-buffered in TMEM (2 x 256 columns).
+//   * warps 2-5: epilogue — tcgen05.ld 32 rows x 32 columns, scale by alpha, zero the strictly
+//     lower triangle, stage in 128B-swizzled smem and add into H with a TMA reduce-add
+//     (cp.reduce.async.bulk.tensor .add), which also clips the ragged edge of H.
+//   * Every mbarrier wait is bounded; on timeout the CTA records GPTQ_ERR_TIMEOUT, leaves its
+//     loops, frees TMEM and returns.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int BOX = 64;                           // 64 bf16 = 128 B inner, 64 tokens outer
+constexpr int BOX_BYTES = BOX * BOX * 2;          // 8 KB
+constexpr int A_BYTES = 2 * BOX_BYTES;            // 16 KB
+constexpr int B_BYTES = 4 * BOX_BYTES;            // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;    // 48 KB
+constexpr int EPI_WARPS = 4;
+constexpr int EPI_TILE_BYTES = 32 * 32 * 4;       // 32 rows x 32 fp32 = 4 KB
+constexpr int EPI_BUFS = 2;
+constexpr int SMEM_DATA = STAGES * STAGE_BYTES + EPI_WARPS * EPI_BUFS * EPI_TILE_BYTES;
+constexpr int SMEM_BYTES = SMEM_DATA + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int THREADS = 192;
+constexpr uint32_t TMEM_COLS = 512;               // two 128 x 256 fp32 accumulators
+constexpr uint32_t IDESC = gptq::instr_desc(/*bf16*/ 1, /*A MN*/ 1, /*B MN*/ 1, BM, BN);
+
+struct SyrkArgs {
+  int d, n_ib, n_jb, n_tiles, n_split, kb_per_split, nkb_total;
+  long long n_units;
+  float alpha;
+  int32_t* status;
+};
+
+// Tile t (0..n_tiles-1) -> (ib, jb): column blocks jb in order, each with the row blocks
+// ib = 0..min(2*jb+1, n_ib-1) that reach the upper triangle.
+__device__ __forceinline__ void tile_coords(int t, int n_ib, int n_jb, int& ib, int& jb) {
+  for (jb = 0; jb < n_jb; ++jb) {
+    int cnt = min(2 * jb + 2, n_ib);
+    if (t < cnt) { ib = t; return; }
+    t -= cnt;
+  }
+  ib = 0;  // unreachable for t < n_tiles
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+syrk_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_x,
+                         const __grid_constant__ CUtensorMap tmap_h, SyrkArgs args) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* stage_base = smem;
+  uint8_t* epi_base = smem + STAGES * STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SMEM_DATA);
+  uint64_t* full = bars;                 // [STAGES]
+  uint64_t* empty = bars + STAGES;       // [STAGES]
+  uint64_t* acc_full = bars + 2 * STAGES;    // [2]
+  uint64_t* acc_empty = bars + 2 * STAGES + 2;  // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* skip_flag = abort_flag + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    *skip_flag = gptq::status_bad(args.status) ? 1 : 0;
+    *abort_flag = 0;
+    for (int s = 0; s < STAGES; ++s) {
+      gptq::mbar_init(&full[s], 1);
+      gptq::mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      gptq::mbar_init(&acc_full[b], 1);
+      gptq::mbar_init(&acc_empty[b], EPI_WARPS);
+    }
+    gptq::fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    gptq::tma_prefetch_desc(&tmap_x);
+    gptq::tma_prefetch_desc(&tmap_h);
+  }
+  if (warp == 1) {
+    gptq::tmem_alloc(tmem_slot, TMEM_COLS);
+    gptq::tmem_relinquish();
+  }
+  gptq::tc_fence_before();
+  __syncthreads();
+  gptq::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const bool skip = *skip_flag != 0;
+
+  if (!skip) {
+    if (warp == 0) {
+      // ------------------------------- TMA producer -------------------------------
+      if (lane == 0) {
+        int stage = 0;
+        uint32_t phase = 0;
+        for (long long u = blockIdx.x; u < args.n_units && !*abort_flag; u += gridDim.x) {
+          const int tile = (int)(u % args.n_tiles), split = (int)(u / args.n_tiles);
+          int ib, jb;
+          tile_coords(tile, args.n_ib, args.n_jb, ib, jb);
+          const int kb0 = split * args.kb_per_split;
+          const int kb1 = min(args.nkb_total, kb0 + args.kb_per_split);
+          for (int kb = kb0; kb < kb1; ++kb) {
+            if (!gptq::mbar_wait(&empty[stage], phase ^ 1, abort_flag)) break;
+            uint8_t* sa = stage_base + stage * STAGE_BYTES;
+            uint8_t* sb = sa + A_BYTES;
+            gptq::mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+            const int t = kb * BK;
+            gptq::tma_load_2d(sa, &tmap_x, &full[stage], ib * BM, t);
+            gptq::tma_load_2d(sa + BOX_BYTES, &tmap_x, &full[stage], ib * BM + BOX, t);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              gptq::tma_load_2d(sb + q * BOX_BYTES, &tmap_x, &full[stage], jb * BN + q * BOX, t);
+            if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          }
+        }
+      }
+    } else if (warp == 1) {
+      // ------------------------------- MMA issuer ---------------------------------
+      if (lane == 0) {
+        int stage = 0;
+        uint32_t phase = 0;
+        int buf = 0;
+        uint32_t acc_phase = 0;
+        for (long long u = blockIdx.x; u < args.n_units && !*abort_flag; u += gridDim.x) {
+          const int split = (int)(u / args.n_tiles);
+          const int kb0 = split * args.kb_per_split;
+          const int kb1 = min(args.nkb_total, kb0 + args.kb_per_split);
+          if (!gptq::mbar_wait(&acc_empty[buf], acc_phase ^ 1, abort_flag)) break;
+          gptq::tc_fence_after();
+          const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
+          bool ok = true;
+          for (int kb = kb0; kb < kb1; ++kb) {
+            if (!gptq::mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+            gptq::tc_fence_after();
+            const uint32_t sa = gptq::smem_u32(stage_base + stage * STAGE_BYTES);
+            const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk) {
+              // MN-major, 128B swizzle: MN atoms (64 elements) every 8 KB (one TMA box),
+              // 8-token K groups every 1 KB; K=16 advances 16 rows = 2 KB.
+              const uint64_t adesc = gptq::smem_desc_sw128(sa + kk * 2048, BOX_BYTES, 1024);
+              const uint64_t bdesc = gptq::smem_desc_sw128(sb + kk * 2048, BOX_BYTES, 1024);
+              gptq::mma_f16(d_tmem, adesc, bdesc, IDESC, (kb > kb0 || kk > 0) ? 1u : 0u);
+            }
+            gptq::mma_commit(&empty[stage]);
+            if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          }
+          if (!ok) break;
+          gptq::mma_commit(&acc_full[buf]);
+          if (++buf == 2) { buf = 0; acc_phase ^= 1; }
+        }
+      }
+    } else {
+      // ------------------------------- epilogue -----------------------------------
+      const int quarter = warp & 3;  // TMEM lanes 32*quarter .. 32*quarter+31
+      uint8_t* my_bufs = epi_base + (warp - 2) * EPI_BUFS * EPI_TILE_BYTES;
+      int buf = 0;
+      uint32_t acc_phase = 0;
+      uint32_t chunk_counter = 0;
+      for (long long u = blockIdx.x; u < args.n_units && !*abort_flag; u += gridDim.x) {
+        const int tile = (int)(u % args.n_tiles);
+        int ib, jb;
+        tile_coords(tile, args.n_ib, args.n_jb, ib, jb);
+        if (!gptq::mbar_wait(&acc_full[buf], acc_phase, abort_flag)) break;
+        gptq::tc_fence_after();
+        const int row0 = ib * BM + quarter * 32;
+        const int row = row0 + lane;
+        const bool rows_live = row0 < args.d;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          const int col0 = jb * BN + c * 32;
+          uint32_t r[32];
+          const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) +
+                                 (uint32_t)(buf * BN + c * 32);
+          gptq::tmem_ld_32x32b_x32(taddr, r);
+          gptq::tmem_ld_wait();
+          // Chunk entirely below the diagonal or outside H: nothing to add.
+          const bool live = rows_live && col0 < args.d && row0 <= col0 + 31;
+          if (!live) continue;
+          uint8_t* sbuf = my_bufs + (chunk_counter & 1) * EPI_TILE_BYTES;
+          if (chunk_counter >= 2) {
+            if (lane == 0) gptq::bulk_wait_read<1>();
+            __syncwarp();
+          }
+          ++chunk_counter;
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4) {
+            float4 v;
+            float* vp = reinterpret_cast<float*>(&v);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int col = col0 + q4 * 4 + e;
+              const float x = __uint_as_float(r[q4 * 4 + e]) * args.alpha;
+              vp[e] = (row <= col) ? x : 0.0f;
+            }
+            // 128B swizzle: 16-byte chunk q4 of row `lane` lives at chunk q4 ^ (lane & 7).
+            *reinterpret_cast<float4*>(sbuf + lane * 128 + ((q4 ^ (lane & 7)) << 4)) = v;
+          }
+          gptq::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            gptq::tma_reduce_add_2d(&tmap_h, sbuf, col0, row0);
+            gptq::bulk_commit();
+          }
+        }
+        gptq::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) gptq::mbar_arrive(&acc_empty[buf]);
+        if (++buf == 2) { buf = 0; acc_phase ^= 1; }
+      }
+      if (lane == 0) gptq::bulk_wait<0>();
+      __syncwarp();
+    }
+  }
+
+  gptq::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) gptq::tmem_dealloc(tmem_base, TMEM_COLS);
+  if (threadIdx.x == 0 && *abort_flag) gptq::set_status(args.status, GPTQ_ERR_TIMEOUT, 1);
+}
+
+__global__ void zero_upper_kernel(float* H, int d, long long ldh) {
+  const long long total = (long long)d * d;
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
+       e += (long long)gridDim.x * blockDim.x) {
+    const int i = (int)(e / d), j = (int)(e % d);
+    if (i <= j) H[i * ldh + j] = 0.0f;
+  }
+}
+
+}  // namespace
+
+namespace gptq_host {
+
+int syrk_bf16_upper(float* H, int d, long long ldh, const void* X, long long n_tokens,
+                    long long ldx, float alpha, int accumulate, int32_t* status,
+                    cudaStream_t stream) {
+  if (!accumulate) {
+    zero_upper_kernel<<<num_sms() * 4, 256, 0, stream>>>(H, d, ldh);
+    if (cudaGetLastError() != cudaSuccess) return GPTQ_ERR_CUDA;
+  }
+  if (n_tokens == 0) return GPTQ_OK;
+
+  CUtensorMap tx, th;
+  if (make_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, X, (uint64_t)d, (uint64_t)n_tokens,
+                   (uint64_t)ldx * 2, BOX, BOX, CU_TENSOR_MAP_SWIZZLE_128B) != 0)
+    return GPTQ_ERR_CUDA;
+  if (make_tmap_2d(&th, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, H, (uint64_t)d, (uint64_t)d,
+                   (uint64_t)ldh * 4, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B) != 0)
+    return GPTQ_ERR_CUDA;
+
+  SyrkArgs a;
+  a.d = d;
+  a.n_ib = (d + BM - 1) / BM;
+  a.n_jb = (d + BN - 1) / BN;
+  a.n_tiles = 0;
+  for (int jb = 0; jb < a.n_jb; ++jb) a.n_tiles += (2 * jb + 2 < a.n_ib) ? 2 * jb + 2 : a.n_ib;
+  a.nkb_total = (int)((n_tokens + BK - 1) / BK);
+  // Split the token range only as far as needed to fill the SMs: pick the split count
+  // (<= 64, every split non-empty) whose last wave is fullest, preferring >= 4 waves.
+  const int sms = num_sms();
+  int best_split = 1;
+  double best_score = -1.0;
+  for (int s = 1; s <= 64 && s <= a.nkb_total; ++s) {
+    const int per = (a.nkb_total + s - 1) / s;
+    const int s_eff = (a.nkb_total + per - 1) / per;
+    if (s_eff != s) continue;
+    const double units = (double)a.n_tiles * s;
+    const double waves = units / sms;
+    const double eff = waves / ceil(waves);
+    const double score = eff - (waves < 4.0 ? 0.25 : 0.0) - 0.002 * s;
+    if (score > best_score) { best_score = score; best_split = s; }
+    if (a.n_tiles >= 8 * sms) break;  // plenty of tiles: no split
+  }
+  a.n_split = best_split;
+  a.kb_per_split = (a.nkb_total + best_split - 1) / best_split;
+  a.n_units = (long long)a.n_tiles * a.n_split;
+  a.alpha = alpha;
+  a.status = status;
+
+  if (cudaFuncSetAttribute(syrk_bf16_tcgen05_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           SMEM_BYTES) != cudaSuccess)
+    return GPTQ_ERR_CUDA;
+  const int grid = (int)(a.n_units < sms ? a.n_units : sms);
+  syrk_bf16_tcgen05_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tx, th, a);
+  return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ERR_CUDA;
+}
+
+}  // namespace gptq_host

@@ -1,0 +1,100 @@
+"""The C ABI library loads, exports every function include/gptq.h declares, and rejects bad
+arguments on the host before touching the GPU (runs without a GPU)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from post_weight_quantization_18_b200 import build
+    path = build.build()
+    return ctypes.CDLL(path)
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "gptq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w]+\s*\*?\s*((?:gptq|rtn)_\w+)\s*\(", src,
+                                 flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    assert declared_functions() == sorted([
+        "gptq_hessian_accumulate", "gptq_pack", "gptq_prepare_hinv", "gptq_quantize_layer",
+        "gptq_status_string", "gptq_workspace_size", "rtn_quantize"])
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_binding_names_match_header():
+    import post_weight_quantization_18_b200 as G
+    assert sorted(G.EXPORTED) == declared_functions()
+    for name in declared_functions():
+        assert callable(getattr(G, name))
+
+
+class P(ctypes.Structure):
+    _fields_ = [("bits", ctypes.c_int32), ("group_size", ctypes.c_int32), ("sym", ctypes.c_int32),
+                ("order", ctypes.c_int32), ("block_size", ctypes.c_int32),
+                ("percdamp", ctypes.c_float)]
+
+
+def test_status_strings(lib):
+    lib.gptq_status_string.restype = ctypes.c_char_p
+    names = {c: lib.gptq_status_string(c).decode() for c in (0, 1, 2, 3, 4, 16, 17, 18, 99)}
+    assert names[0] == "GPTQ_OK" and names[16] == "GPTQ_ERR_NOT_SPD"
+    assert names[18] == "GPTQ_ERR_TIMEOUT" and names[99] == "GPTQ_ERR_UNKNOWN"
+
+
+def test_workspace_size(lib):
+    lib.gptq_workspace_size.restype = ctypes.c_size_t
+    lib.gptq_workspace_size.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.POINTER(P)]
+    ok = P(4, 128, 0, 0, 128, 0.01)
+    assert lib.gptq_workspace_size(4096, 4096, ctypes.byref(ok)) == 2 * 4096 * 4096 * 4
+    act = P(3, 128, 0, 1, 128, 0.01)
+    assert lib.gptq_workspace_size(4096, 4096, ctypes.byref(act)) == 2 * 4096 * 4096 * 4 + 4096 * 4096
+    for bad in (P(5, 128, 0, 0, 128, 0.01), P(4, 96, 0, 0, 128, 0.01), P(4, 128, 0, 0, 64, 0.01),
+                P(4, 128, 2, 0, 128, 0.01), P(4, 128, 0, 3, 128, 0.01), P(4, 6, 0, 0, 128, 0.01),
+                P(4, 128, 0, 0, 128, -1.0)):
+        assert lib.gptq_workspace_size(4096, 4096, ctypes.byref(bad)) == 0
+    assert lib.gptq_workspace_size(0, 4096, ctypes.byref(ok)) == 0
+
+
+def test_invalid_arguments_rejected_on_host(lib):
+    V = ctypes.c_void_p
+    fake = V(0x1000)  # never dereferenced: every call below fails its host-side checks
+    lib.gptq_hessian_accumulate.argtypes = [V, ctypes.c_int64, ctypes.c_int64, V, ctypes.c_int,
+                                            ctypes.c_int64, ctypes.c_int64, ctypes.c_float,
+                                            ctypes.c_int, V, V]
+    assert lib.gptq_hessian_accumulate(None, 64, 64, fake, 0, 10, 64, 2.0, 0, None, None) == 1
+    assert lib.gptq_hessian_accumulate(fake, 64, 32, fake, 0, 10, 64, 2.0, 0, None, None) == 1
+    assert lib.gptq_hessian_accumulate(fake, 64, 64, fake, 0, 10, 32, 2.0, 0, None, None) == 1
+    assert lib.gptq_hessian_accumulate(fake, 64, 64, fake, 7, 10, 64, 2.0, 0, None, None) == 2
+    assert lib.gptq_hessian_accumulate(fake, 64, 64, fake, 0, 10, 66, 2.0, 0, None, None) == 1
+    p = P(4, 128, 0, 0, 128, 0.01)
+    lib.gptq_quantize_layer.argtypes = [V, ctypes.c_int, ctypes.c_int64, ctypes.c_int64,
+                                        ctypes.c_int64, V, V, V, ctypes.POINTER(P), V, V, V, V, V,
+                                        ctypes.c_size_t, V, V]
+    args = lambda d_in, ws_bytes: (fake, 0, d_in, 16, d_in, fake, fake, fake, ctypes.byref(p), fake,
+                                   fake, fake, fake, fake, ws_bytes, None, None)
+    assert lib.gptq_quantize_layer(*args(100, 1 << 30)) == 1      # d_in not a multiple of 128
+    assert lib.gptq_quantize_layer(*args(256, 16)) == 3           # workspace too small
+    lib.gptq_pack.argtypes = [V, ctypes.c_int64, ctypes.c_int64, ctypes.c_int, V, V,
+                              ctypes.c_int64, V, V, V, V]
+    assert lib.gptq_pack(fake, 4, 64, 5, fake, fake, 1, fake, fake, fake, None) == 1
+    lib.rtn_quantize.argtypes = [V, ctypes.c_int, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                 ctypes.POINTER(P), V, V, V, V]
+    bad_g = P(4, 100, 0, 0, 128, 0.01)
+    assert lib.rtn_quantize(fake, 0, 256, 4, 256, ctypes.byref(bad_g), fake, fake, fake, None) == 1
+    lib.gptq_prepare_hinv.argtypes = [V, ctypes.c_int64, ctypes.POINTER(P), V, V, V, V,
+                                      ctypes.c_size_t, V, V]
+    assert lib.gptq_prepare_hinv(fake, 64, ctypes.byref(p), fake, None, fake, None, 0, None,
+                                 None) == 1

@@ -1,0 +1,106 @@
+"""GPU parity: the full layer (Hessian -> prepare -> sweep) against the oracle, and RTN/pack
+bit-exactness."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_util import compare_with_oracle, f64, gpu_pipeline, make_inputs
+from oracle import pack as pk
+from oracle import quantizer as qz
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("n,d,N,bits,g,sym,half", [
+    (300, 640, 6000, 4, 128, False, False),     # several leaves, ragged rows
+    (37, 256, 3000, 4, 128, False, True),       # fewer rows than one CTA
+    (256, 512, 5000, 3, 128, False, False),     # 3-bit
+    (200, 384, 4000, 4, 64, False, False),      # two groups per block
+    (128, 256, 3000, 4, 32, True, False),       # symmetric groups
+    (160, 1024, 9000, 4, -1, True, True),       # one symmetric scale per row
+    (96, 1280, 15000, 2, 128, False, False),    # 2-bit
+])
+def test_layer_matches_oracle(n, d, N, bits, g, sym, half):
+    W, X = make_inputs(n, d, N, seed=n + d + bits, half_normal=half)
+    compare_with_oracle(W, X, bits=bits, group_size=g, sym=sym)
+
+
+def test_act_order_given_perm_matches_oracle():
+    W, X = make_inputs(200, 512, 6000, seed=77)
+    compare_with_oracle(W, X, bits=3, group_size=128, act_order=True, given_perm=True)
+
+
+def test_act_order_desc_act_on_gpu():
+    W, X = make_inputs(128, 384, 5000, seed=78)
+    compare_with_oracle(W, X, bits=4, group_size=128, act_order=True, given_perm=False,
+                        code_agree=0.99, err_rtol=5e-3)
+
+
+def test_fp32_small_workload():
+    """The small fp32 layer (256 x 256, 2048 tokens, lognormal(0, 0.5) channels)."""
+    import layer_inputs as li
+    wl = li.WORKLOADS["tiny_256"]
+    X = wl.acts[0].make()
+    W = wl.linears[0].make()
+    compare_with_oracle(W, X, bits=4, group_size=128)
+
+
+@pytest.mark.parametrize("g,sym", [(128, False), (64, False), (-1, True)])
+def test_identity_hessian_gives_rtn(g, sym):
+    """H = I: GPU GPTQ codes == GPU RTN codes == oracle RTN codes (bit for bit)."""
+    import post_weight_quantization_18_b200 as G
+    W, _ = make_inputs(256, 256, 8, seed=5, w_dtype=torch.float32)
+    res = gpu_pipeline(W, H=np.eye(256), bits=4, group_size=g, sym=sym)
+    codes_rtn, s_rtn, z_rtn = G.rtn(W.cuda(), 4, g, sym)
+    ora = oracle.rtn_layer(W.numpy(), 4, g, sym)
+    np.testing.assert_array_equal(res["codes"], codes_rtn.cpu().numpy())
+    np.testing.assert_array_equal(codes_rtn.cpu().numpy(), ora["codes"])
+    np.testing.assert_array_equal(s_rtn.cpu().numpy(), ora["S"])
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("bits,g,sym", [(4, 128, False), (3, 128, False), (4, -1, True),
+                                        (8, 64, True), (4, 100, False)])
+def test_rtn_bit_exact(dtype, bits, g, sym):
+    import post_weight_quantization_18_b200 as G
+    W, _ = make_inputs(333, 1200, 8, seed=9, w_dtype=dtype)
+    codes, s, z = G.rtn(W.cuda(), bits, g, sym)
+    ora = oracle.rtn_layer(W.float().numpy(), bits, g, sym)
+    np.testing.assert_array_equal(codes.cpu().numpy(), ora["codes"])
+    np.testing.assert_array_equal(s.cpu().numpy(), ora["S"])
+    np.testing.assert_array_equal(z.cpu().numpy(), ora["Z"])
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+@pytest.mark.parametrize("d", [128, 200, 4096])
+def test_pack_bit_exact(bits, d):
+    import post_weight_quantization_18_b200 as G
+    rng = np.random.default_rng(bits * 31 + d)
+    n, Gn = 57, 3
+    codes = rng.integers(0, 2 ** bits, (n, d), dtype=np.uint8)
+    S = rng.lognormal(-5, 2, (n, Gn)).astype(np.float32)
+    Z = rng.integers(0, 2 ** bits, (n, Gn)).astype(np.float32)
+    qw = torch.empty((n, (d * bits + 31) // 32), dtype=torch.int32, device="cuda")
+    s16 = torch.empty((n, Gn), dtype=torch.int16, device="cuda")
+    z16 = torch.empty((n, Gn), dtype=torch.int16, device="cuda")
+    G.gptq_pack(torch.from_numpy(codes).cuda(), bits, torch.from_numpy(S).cuda(),
+                torch.from_numpy(Z).cuda(), qw, s16, z16)
+    ow, os16, oz16 = pk.pack(codes, S, Z, bits)
+    np.testing.assert_array_equal(qw.cpu().numpy().view(np.uint32), ow)
+    np.testing.assert_array_equal(s16.cpu().numpy().view(np.uint16), os16)
+    np.testing.assert_array_equal(z16.cpu().numpy().view(np.uint16), oz16)
+
+
+def test_gptq_beats_rtn_on_gpu():
+    W, X = make_inputs(256, 512, 8000, seed=3)
+    W64, X64 = f64(W), f64(X)
+    from oracle import error as er
+    from oracle import hessian as hs
+    H64 = hs.hessian(X64)
+    res = gpu_pipeline(W, X)
+    R = oracle.rtn_layer(W64, 4, 128, False)
+    e_g = er.layer_error(W64, er.dequant_matrix(res["codes"], res["S"], res["Z"], res["g_idx"]),
+                         H64)
+    e_r = er.layer_error(W64, er.dequant_matrix(R["codes"], R["S"], R["Z"], R["g_idx"]), H64)
+    assert e_g < 0.9 * e_r
