@@ -261,6 +261,25 @@ def config_dict(args, wl, world):
 
 
 # ------------------------------------------------------------------------------------------
+# Multi-rank plumbing (independent layers per rank; only timing crosses ranks)
+# ------------------------------------------------------------------------------------------
+
+def max_over_ranks(values, device):
+    """Element-wise max over all ranks of a few host floats (identity when not distributed)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.cpu().tolist()
+
+
+def rank_seed_offset(rank):
+    """Each rank quantizes its own layer: same shapes and distributions, disjoint seeds."""
+    return 100000 * rank
+
+
+# ------------------------------------------------------------------------------------------
 # Our arm
 # ------------------------------------------------------------------------------------------
 
@@ -287,6 +306,9 @@ def run_ours(args):
     n, d, N = lin.d_out, lin.d_in, act.n_tokens
 
     # Inputs: pinned host copies (for the end-to-end measurement) and device copies.
+    import dataclasses
+    act = dataclasses.replace(act, seed=act.seed + rank_seed_offset(rank))
+    lin = dataclasses.replace(lin, seed=lin.seed + rank_seed_offset(rank))
     Xh = torch.empty((N, d), dtype=torch.bfloat16).pin_memory()
     act.make(out=Xh)
     Wh = lin.make().pin_memory()
@@ -376,10 +398,7 @@ def run_ours(args):
     total_s = sum(step_ms) / 1e3
     e2e_ms = [a.elapsed_time(b) for a, b in e2e_ev]
     e2e_total_s = sum(e2e_ms) / 1e3
-    t = torch.tensor([total_s, e2e_total_s], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_s, e2e_total_s = t.tolist()
+    total_s, e2e_total_s = max_over_ranks([total_s, e2e_total_s], dev)
 
     if rank == 0:
         hbm, bf16, peak_kind = peaks()

@@ -152,7 +152,7 @@ size_t gptq_workspace_size(int64_t d_out, int64_t d_in, const gptq_params* p) {
 int gptq_hessian_accumulate(float* H, int64_t d_in, int64_t ldh, const void* X, int x_dtype,
                             int64_t n_tokens, int64_t ldx, float alpha, int accumulate,
                             int32_t* dev_status, gptq_stream_t stream) {
-  if (H == nullptr || X == nullptr || d_in < 1 || d_in > (1 << 30) || n_tokens < 0 ||
+  if (H == nullptr || (X == nullptr && n_tokens > 0) || d_in < 1 || d_in > (1 << 30) || n_tokens < 0 ||
       n_tokens > (int64_t(1) << 31) - 1 || ldx < d_in || ldh < d_in)
     return GPTQ_ERR_INVALID_ARG;
   if (accumulate != 0 && accumulate != 1) return GPTQ_ERR_INVALID_ARG;
@@ -160,7 +160,7 @@ int gptq_hessian_accumulate(float* H, int64_t d_in, int64_t ldh, const void* X, 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (x_dtype == GPTQ_BF16) {
     // TMA: 16-byte aligned bases and row strides.
-    if (!aligned(X, 16) || (ldx % 8) != 0 || !aligned(H, 16) || (ldh % 4) != 0)
+    if ((n_tokens > 0 && (!aligned(X, 16) || (ldx % 8) != 0)) || !aligned(H, 16) || (ldh % 4) != 0)
       return GPTQ_ERR_INVALID_ARG;
     return gptq_host::syrk_bf16_upper(H, (int)d_in, ldh, X, n_tokens, ldx, alpha, accumulate,
                                       dev_status, s);

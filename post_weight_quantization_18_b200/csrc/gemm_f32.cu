@@ -102,15 +102,32 @@ gemm_f32_simt_kernel(int M, int N, int K, float alpha, const float* __restrict__
 
 namespace gptq_host {
 
-int gemm_f32(int M, int N, int K, float alpha, const float* A, long long lda, bool transA,
-             const float* B, long long ldb, bool transB, float beta, float* C, long long ldc,
-             bool upper_only, const int32_t* status, cudaStream_t stream) {
+// CUDA-core GEMM: used only where TMA cannot address the operands (row strides or bases not
+// 16-byte aligned) and for K = 0; everything else goes to the tcgen05 3xTF32 kernel.
+int gemm_f32_simt(int M, int N, int K, float alpha, const float* A, long long lda, bool transA,
+                  const float* B, long long ldb, bool transB, float beta, float* C, long long ldc,
+                  bool upper_only, const int32_t* status, cudaStream_t stream) {
   if (M <= 0 || N <= 0) return 0;
   dim3 grid((N + TN - 1) / TN, (M + TM - 1) / TM);
   gemm_f32_simt_kernel<<<grid, THREADS, 0, stream>>>(M, N, K, alpha, A, lda, transA ? 1 : 0, B,
                                                      ldb, transB ? 1 : 0, beta, C, ldc,
                                                      upper_only ? 1 : 0, status);
   return cudaGetLastError() == cudaSuccess ? 0 : GPTQ_ERR_CUDA;
+}
+
+}  // namespace gptq_host
+
+namespace gptq_host {
+
+int gemm_f32(int M, int N, int K, float alpha, const float* A, long long lda, bool transA,
+             const float* B, long long ldb, bool transB, float beta, float* C, long long ldc,
+             bool upper_only, const int32_t* status, cudaStream_t stream) {
+  if (M <= 0 || N <= 0) return 0;
+  if (gemm_tf32x3_supported(M, N, K, A, lda, B, ldb, C, ldc))
+    return gemm_tf32x3(M, N, K, alpha, A, lda, transA, B, ldb, transB, beta, C, ldc, upper_only,
+                       status, stream);
+  return gemm_f32_simt(M, N, K, alpha, A, lda, transA, B, ldb, transB, beta, C, ldc, upper_only,
+                       status, stream);
 }
 
 }  // namespace gptq_host

@@ -1,0 +1,332 @@
+// gemm_tf32x3.cu — C = alpha * op(A) op(B) + beta * C in fp32 on tcgen05 tensor cores, with
+// fp32-level accuracy from the 3xTF32 split: x = x_hi + x_lo where x_hi is x with the low 13
+// mantissa bits cleared (exactly representable in tf32) and x_lo = x - x_hi (exact in fp32);
+// a*b ~= a_hi*b_hi + a_hi*b_lo + a_lo*b_hi (the dropped a_lo*b_lo term is ~2^-22 relative).
+//
+// Serves the lazy block updates of the sweep ("GPTQ: Mathematical Foundations ...", §2 Lazy
+// Batch Updates: W[:, F] -= Err_B U[B, F]), the GEMM steps of the U recursion and the Hessian of
+// fp32 calibration inputs.
+//
+// Layout: fp32 row-major operands in global memory, each either K-major (contiguous along K) or
+// MN-major (contiguous along M resp. N); TMA brings 128-byte-swizzled tiles into shared memory.
+// One CTA per SM (persistent), 128 x 128 output tiles, 32-wide K blocks, 3-stage ring.
+//   warp 0      TMA producer
+//   warp 1      TMEM owner + MMA issuer: per 8-wide K step three tcgen05.mma kind::tf32
+//   warps 2-5   converters: split each landed tile in place into hi and a separate lo copy
+//   warps 6-9   epilogue: tcgen05.ld, alpha/beta, masked stores (double-buffered accumulators)
+// Every mbarrier wait is bounded (GPTQ_ERR_TIMEOUT on expiry).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace {
+
+constexpr int BM = 128, BN = 128, BK = 32, STAGES = 3;
+constexpr int TILE_BYTES = 128 * BK * 4;              // 16 KB: one operand tile (128 x 32 fp32)
+constexpr int STAGE_BYTES = 4 * TILE_BYTES;           // A, A_lo, B, B_lo
+constexpr int SMEM_DATA = STAGES * STAGE_BYTES;       // 192 KB
+constexpr int SMEM_BYTES = SMEM_DATA + 1024 + 256;
+constexpr int THREADS = 320;
+constexpr int CONV_WARP0 = 2, N_CONV = 4, EPI_WARP0 = 6, N_EPI = 4;
+constexpr uint32_t TMEM_COLS = 256;                   // two 128 x 128 fp32 accumulators
+
+struct GemmArgs {
+  int M, N, K;
+  float alpha, beta;
+  float* C;
+  long long ldc;
+  int a_mn, b_mn;      // 1: operand is MN-major in memory
+  int upper_only;
+  int tiles_m, tiles_n, n_tiles;
+  const int32_t* status;
+  int32_t* status_w;
+};
+
+// Shared-memory descriptor of one operand tile at K offset kk (in units of 8 elements).
+// K-major: rows of 128 B (32 fp32 of K) in 8-row swizzle atoms (SBO 1 KB); K steps move 32 B.
+// MN-major: four 32-element MN atoms of BK rows each (LBO 4 KB), 8-row K atoms (SBO 1 KB);
+// K steps move 8 rows = 1 KB.
+__device__ __forceinline__ uint64_t op_desc(uint32_t base, int mn_major, int kk) {
+  if (mn_major) return gptq::smem_desc_sw128(base + kk * 1024, 4096, 1024);
+  return gptq::smem_desc_sw128(base + kk * 32, 16, 1024);
+}
+
+__device__ __forceinline__ void tile_of(int t, const GemmArgs& a, int& tm, int& tn) {
+  tm = t / a.tiles_n;
+  tn = t % a.tiles_n;
+}
+
+__device__ __forceinline__ bool tile_live(int tm, int tn, const GemmArgs& a) {
+  return !a.upper_only || (tm * BM <= tn * BN + BN - 1);
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   GemmArgs args) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SMEM_DATA);
+  uint64_t* full = bars;                       // TMA landed        [STAGES]
+  uint64_t* conv = bars + STAGES;              // split done        [STAGES]
+  uint64_t* empty = bars + 2 * STAGES;         // MMA consumed      [STAGES]
+  uint64_t* acc_full = bars + 3 * STAGES;      // [2]
+  uint64_t* acc_empty = bars + 3 * STAGES + 2; // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * STAGES + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* skip_flag = abort_flag + 1;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    *skip_flag = gptq::status_bad(args.status) ? 1 : 0;
+    *abort_flag = 0;
+    for (int s = 0; s < STAGES; ++s) {
+      gptq::mbar_init(&full[s], 1);
+      gptq::mbar_init(&conv[s], N_CONV);
+      gptq::mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      gptq::mbar_init(&acc_full[b], 1);
+      gptq::mbar_init(&acc_empty[b], N_EPI);
+    }
+    gptq::fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    gptq::tma_prefetch_desc(&tmA);
+    gptq::tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    gptq::tmem_alloc(tmem_slot, TMEM_COLS);
+    gptq::tmem_relinquish();
+  }
+  gptq::tc_fence_before();
+  __syncthreads();
+  gptq::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int nkb = (args.K + BK - 1) / BK;
+
+  if (!*skip_flag) {
+    if (warp == 0) {
+      if (lane == 0) {  // ---------------- TMA producer ----------------
+        int stage = 0;
+        uint32_t phase = 0;
+        for (int t = blockIdx.x; t < args.n_tiles && !*abort_flag; t += gridDim.x) {
+          int tm, tn;
+          tile_of(t, args, tm, tn);
+          if (!tile_live(tm, tn, args)) continue;
+          for (int kb = 0; kb < nkb; ++kb) {
+            if (!gptq::mbar_wait(&empty[stage], phase ^ 1, abort_flag)) break;
+            uint8_t* sa = smem + stage * STAGE_BYTES;
+            uint8_t* sb = sa + 2 * TILE_BYTES;
+            gptq::mbar_arrive_expect_tx(&full[stage], 2 * TILE_BYTES);
+            const int k0 = kb * BK;
+            if (args.a_mn) {
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                gptq::tma_load_2d(sa + q * 4096, &tmA, &full[stage], tm * BM + 32 * q, k0);
+            } else {
+              gptq::tma_load_2d(sa, &tmA, &full[stage], k0, tm * BM);
+            }
+            if (args.b_mn) {
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                gptq::tma_load_2d(sb + q * 4096, &tmB, &full[stage], tn * BN + 32 * q, k0);
+            } else {
+              gptq::tma_load_2d(sb, &tmB, &full[stage], k0, tn * BN);
+            }
+            if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          }
+        }
+      }
+    } else if (warp == 1) {
+      if (lane == 0) {  // ---------------- MMA issuer ----------------
+        const uint32_t idesc = gptq::instr_desc(/*tf32*/ 2, args.a_mn, args.b_mn, BM, BN);
+        int stage = 0;
+        uint32_t phase = 0;
+        int buf = 0;
+        uint32_t acc_phase = 0;
+        for (int t = blockIdx.x; t < args.n_tiles && !*abort_flag; t += gridDim.x) {
+          int tm, tn;
+          tile_of(t, args, tm, tn);
+          if (!tile_live(tm, tn, args)) continue;
+          if (!gptq::mbar_wait(&acc_empty[buf], acc_phase ^ 1, abort_flag)) break;
+          gptq::tc_fence_after();
+          const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
+          bool ok = true;
+          for (int kb = 0; kb < nkb; ++kb) {
+            if (!gptq::mbar_wait(&conv[stage], phase, abort_flag)) { ok = false; break; }
+            gptq::tc_fence_after();
+            const uint32_t a_hi = gptq::smem_u32(smem + stage * STAGE_BYTES);
+            const uint32_t a_lo = a_hi + TILE_BYTES;
+            const uint32_t b_hi = a_hi + 2 * TILE_BYTES;
+            const uint32_t b_lo = a_hi + 3 * TILE_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < BK / 8; ++kk) {
+              const uint64_t dah = op_desc(a_hi, args.a_mn, kk), dal = op_desc(a_lo, args.a_mn, kk);
+              const uint64_t dbh = op_desc(b_hi, args.b_mn, kk), dbl = op_desc(b_lo, args.b_mn, kk);
+              gptq::mma_tf32(d_tmem, dah, dbl, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+              gptq::mma_tf32(d_tmem, dal, dbh, idesc, 1u);
+              gptq::mma_tf32(d_tmem, dah, dbh, idesc, 1u);
+            }
+            gptq::mma_commit(&empty[stage]);
+            if (++stage == STAGES) { stage = 0; phase ^= 1; }
+          }
+          if (!ok) break;
+          gptq::mma_commit(&acc_full[buf]);
+          if (++buf == 2) { buf = 0; acc_phase ^= 1; }
+        }
+      }
+    } else if (warp < EPI_WARP0) {
+      // ---------------- converters: x -> (hi in place, lo copy) ----------------
+      const int ct = threadIdx.x - CONV_WARP0 * 32;  // 0..127
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int t = blockIdx.x; t < args.n_tiles && !*abort_flag; t += gridDim.x) {
+        int tm, tn;
+        tile_of(t, args, tm, tn);
+        if (!tile_live(tm, tn, args)) continue;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!gptq::mbar_wait(&full[stage], phase, abort_flag)) break;
+          uint8_t* st = smem + stage * STAGE_BYTES;
+#pragma unroll
+          for (int op = 0; op < 2; ++op) {
+            float4* hi = reinterpret_cast<float4*>(st + op * 2 * TILE_BYTES);
+            float4* lo = reinterpret_cast<float4*>(st + op * 2 * TILE_BYTES + TILE_BYTES);
+#pragma unroll 4
+            for (int e = ct; e < TILE_BYTES / 16; e += N_CONV * 32) {
+              float4 x = hi[e], h, l;
+              h.x = __uint_as_float(__float_as_uint(x.x) & 0xFFFFE000u);
+              h.y = __uint_as_float(__float_as_uint(x.y) & 0xFFFFE000u);
+              h.z = __uint_as_float(__float_as_uint(x.z) & 0xFFFFE000u);
+              h.w = __uint_as_float(__float_as_uint(x.w) & 0xFFFFE000u);
+              l.x = x.x - h.x; l.y = x.y - h.y; l.z = x.z - h.z; l.w = x.w - h.w;
+              hi[e] = h;
+              lo[e] = l;
+            }
+          }
+          gptq::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) gptq::mbar_arrive(&conv[stage]);
+          if (++stage == STAGES) { stage = 0; phase ^= 1; }
+        }
+      }
+    } else {
+      // ---------------- epilogue ----------------
+      const int quarter = warp & 3;
+      int buf = 0;
+      uint32_t acc_phase = 0;
+      for (int t = blockIdx.x; t < args.n_tiles && !*abort_flag; t += gridDim.x) {
+        int tm, tn;
+        tile_of(t, args, tm, tn);
+        if (!tile_live(tm, tn, args)) continue;
+        if (!gptq::mbar_wait(&acc_full[buf], acc_phase, abort_flag)) break;
+        gptq::tc_fence_after();
+        const int row = tm * BM + quarter * 32 + lane;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t r[32];
+          __syncwarp();  // tcgen05.ld is warp-collective: reconverge before every load
+          gptq::tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(quarter * 32) << 16) +
+                                       (uint32_t)(buf * BN + c * 32),
+                                   r);
+          gptq::tmem_ld_wait();
+          const int col0 = tn * BN + c * 32;
+          if (row < args.M && col0 < args.N) {
+            float* crow = args.C + (long long)row * args.ldc;
+            const bool full_vec = (col0 + 32 <= args.N) && (!args.upper_only || row <= col0);
+            if (full_vec) {
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                float4* p = reinterpret_cast<float4*>(crow + col0 + 4 * q);
+                float4 o;
+                o.x = args.alpha * __uint_as_float(r[4 * q + 0]);
+                o.y = args.alpha * __uint_as_float(r[4 * q + 1]);
+                o.z = args.alpha * __uint_as_float(r[4 * q + 2]);
+                o.w = args.alpha * __uint_as_float(r[4 * q + 3]);
+                if (args.beta != 0.f) {
+                  const float4 old = *p;
+                  o.x = fmaf(args.beta, old.x, o.x);
+                  o.y = fmaf(args.beta, old.y, o.y);
+                  o.z = fmaf(args.beta, old.z, o.z);
+                  o.w = fmaf(args.beta, old.w, o.w);
+                }
+                *p = o;
+              }
+            } else {
+#pragma unroll
+              for (int e = 0; e < 32; ++e) {
+                const int col = col0 + e;
+                if (col >= args.N || (args.upper_only && row > col)) continue;
+                float o = args.alpha * __uint_as_float(r[e]);
+                if (args.beta != 0.f) o = fmaf(args.beta, crow[col], o);
+                crow[col] = o;
+              }
+            }
+          }
+        }
+        gptq::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) gptq::mbar_arrive(&acc_empty[buf]);
+        if (++buf == 2) { buf = 0; acc_phase ^= 1; }
+      }
+    }
+  }
+
+  gptq::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) gptq::tmem_dealloc(tmem_base, TMEM_COLS);
+  if (threadIdx.x == 0 && *abort_flag) gptq::set_status(args.status_w, GPTQ_ERR_TIMEOUT, 2);
+}
+
+inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+namespace gptq_host {
+
+bool gemm_tf32x3_supported(int M, int N, int K, const float* A, long long lda, const float* B,
+                           long long ldb, const float* C, long long ldc) {
+  return M > 0 && N > 0 && K > 0 && al16(A) && al16(B) && al16(C) && (lda % 4) == 0 &&
+         (ldb % 4) == 0 && (ldc % 4) == 0;
+}
+
+// op(A) is M x K: transA=false -> A[m*lda + k] (K-major); transA=true -> A[k*lda + m] (MN-major).
+// op(B) is K x N: transB=false -> B[k*ldb + n] (MN-major); transB=true -> B[n*ldb + k] (K-major).
+int gemm_tf32x3(int M, int N, int K, float alpha, const float* A, long long lda, bool transA,
+                const float* B, long long ldb, bool transB, float beta, float* C, long long ldc,
+                bool upper_only, const int32_t* status, cudaStream_t stream) {
+  CUtensorMap ta, tb;
+  const CUtensorMapDataType f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
+  int rc;
+  if (transA)  // MN-major: inner = M
+    rc = make_tmap_2d(&ta, f32, 4, A, (uint64_t)M, (uint64_t)K, (uint64_t)lda * 4, 32, BK, sw);
+  else         // K-major: inner = K
+    rc = make_tmap_2d(&ta, f32, 4, A, (uint64_t)K, (uint64_t)M, (uint64_t)lda * 4, BK, BM, sw);
+  if (rc) return GPTQ_ERR_CUDA;
+  if (!transB)  // MN-major: inner = N
+    rc = make_tmap_2d(&tb, f32, 4, B, (uint64_t)N, (uint64_t)K, (uint64_t)ldb * 4, 32, BK, sw);
+  else          // K-major: inner = K
+    rc = make_tmap_2d(&tb, f32, 4, B, (uint64_t)K, (uint64_t)N, (uint64_t)ldb * 4, BK, BN, sw);
+  if (rc) return GPTQ_ERR_CUDA;
+  GemmArgs a;
+  a.M = M; a.N = N; a.K = K;
+  a.alpha = alpha; a.beta = beta;
+  a.C = C; a.ldc = ldc;
+  a.a_mn = transA ? 1 : 0;
+  a.b_mn = transB ? 0 : 1;
+  a.upper_only = upper_only ? 1 : 0;
+  a.tiles_m = (M + BM - 1) / BM;
+  a.tiles_n = (N + BN - 1) / BN;
+  a.n_tiles = a.tiles_m * a.tiles_n;
+  a.status = status;
+  a.status_w = const_cast<int32_t*>(status);
+  if (cudaFuncSetAttribute(gemm_tf32x3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           SMEM_BYTES) != cudaSuccess)
+    return GPTQ_ERR_CUDA;
+  const int sms = num_sms();
+  const int grid = a.n_tiles < sms ? a.n_tiles : sms;
+  gemm_tf32x3_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(ta, tb, a);
+  return cudaGetLastError() == cudaSuccess ? 0 : GPTQ_ERR_CUDA;
+}
+
+}  // namespace gptq_host

@@ -120,8 +120,12 @@ __global__ void zero_lower_kernel(float* U, int d) {
 }
 
 // Base block (n <= 128): H_d block (upper triangle, ld) -> U block = V^-1 where H_d = V V^T.
-// Right-looking Cholesky from the last column, then V^-1 by the same sweep order applied to
-// the identity. Writes the whole n x n U block (zeros below the diagonal).
+// Phase 1 (Cholesky from the last column), step j: V_jj = sqrt(a_jj), V_ij = a_ij / V_jj, and the
+// leading block a_ik -= V_ij V_kj (i <= k < j). Phase 2 (U = V^-1, back substitution on all
+// columns at once), step i: row i of U = r_i / V_ii (written straight to global memory, it is
+// final) and r_kc -= V_ki U_ic for k < i, c >= i, starting from r = I. Every step reads only a
+// column (phase 1) or a row (phase 2) that the step itself does not write, so one barrier per
+// step suffices. Thread (ty, tx) of the 16 x 32 layout owns rows ty + 16a and columns = tx mod 32.
 constexpr int BASE_THREADS = 512;
 constexpr int BASE_LD = gptq_host::kPrepBase + 1;
 
@@ -129,55 +133,50 @@ __global__ void __launch_bounds__(BASE_THREADS)
 base_block_kernel(float* __restrict__ Hblk, float* __restrict__ Ublk, int n, int ld, int index0,
                   int32_t* status) {
   extern __shared__ float sm[];
-  float* a = sm;                          // [128][129]: V (upper) after the factorization
-  float* r = sm + gptq_host::kPrepBase * BASE_LD;  // [128][129]: U = V^-1
+  float* a = sm;                                   // working matrix, then r
+  float* v = sm + gptq_host::kPrepBase * BASE_LD;  // V (upper)
   __shared__ int bad;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, tx = tid & 31, ty = tid >> 5;
   if (tid == 0) bad = gptq::status_bad(status) ? 1 : 0;
+  for (int i = ty; i < n; i += 16)
+    for (int k = tx; k < n; k += 32) a[i * BASE_LD + k] = (i <= k) ? Hblk[(long long)i * ld + k] : 0.f;
   __syncthreads();
   if (bad) return;
-  for (int e = tid; e < n * n; e += BASE_THREADS) {
-    const int i = e / n, k = e % n;
-    a[i * BASE_LD + k] = (i <= k) ? Hblk[(long long)i * ld + k] : 0.f;
-    r[i * BASE_LD + k] = (i == k) ? 1.f : 0.f;
-  }
-  __syncthreads();
-  // V: for j = n-1 .. 0: V_jj = sqrt(a_jj), V_ij = a_ij / V_jj (i < j),
-  // a_ik -= V_ij V_kj for i <= k < j.
   for (int j = n - 1; j >= 0; --j) {
     const float piv = a[j * BASE_LD + j];
-    if (!(piv > 0.f) || !isfinite(piv)) {
+    if (!(piv > 0.f) || !isfinite(piv)) {  // uniform: all threads read the same pivot
       if (tid == 0) gptq::set_status(status, GPTQ_ERR_NOT_SPD, index0 + j);
-      return;  // uniform: every thread read the same pivot
+      return;
     }
     const float vjj = sqrtf(piv);
     const float inv = 1.0f / vjj;
-    __syncthreads();
-    for (int i = tid; i <= j; i += BASE_THREADS)
-      a[i * BASE_LD + j] = (i == j) ? vjj : a[i * BASE_LD + j] * inv;
-    __syncthreads();
-    const int m = j;  // leading block 0..j-1
-    for (int e = tid; e < m * m; e += BASE_THREADS) {
-      const int i = e / m, k = e % m;
-      if (i <= k) a[i * BASE_LD + k] = fmaf(-a[i * BASE_LD + j], a[k * BASE_LD + j], a[i * BASE_LD + k]);
+    if (ty == 0) {
+      for (int i = tx; i < j; i += 32) v[i * BASE_LD + j] = a[i * BASE_LD + j] * inv;
+      if (tx == 0) v[j * BASE_LD + j] = vjj;
+    }
+    for (int i = ty; i < j; i += 16) {
+      const float vij = a[i * BASE_LD + j] * inv;
+      for (int k = i + ((tx - i) & 31); k < j; k += 32)
+        a[i * BASE_LD + k] = fmaf(-vij, a[k * BASE_LD + j] * inv, a[i * BASE_LD + k]);
     }
     __syncthreads();
   }
-  // U = V^-1 by back substitution on all columns at once: for i = n-1 .. 0:
-  // row i of U = r_i / V_ii; r_k -= V_ki * U_i for k < i (r starts as the identity).
+  for (int i = ty; i < n; i += 16)
+    for (int k = tx; k < n; k += 32) {
+      a[i * BASE_LD + k] = (i == k) ? 1.f : 0.f;
+      if (k < i) Ublk[(long long)i * ld + k] = 0.f;
+    }
+  __syncthreads();
   for (int i = n - 1; i >= 0; --i) {
-    const float inv = 1.0f / a[i * BASE_LD + i];
-    for (int k = tid; k < n; k += BASE_THREADS) r[i * BASE_LD + k] *= inv;
-    __syncthreads();
-    for (int e = tid; e < i * n; e += BASE_THREADS) {
-      const int k = e / n, c = e % n;
-      r[k * BASE_LD + c] = fmaf(-a[k * BASE_LD + i], r[i * BASE_LD + c], r[k * BASE_LD + c]);
+    const float inv = 1.0f / v[i * BASE_LD + i];
+    if (ty == 0)
+      for (int c = i + tx; c < n; c += 32) Ublk[(long long)i * ld + c] = a[i * BASE_LD + c] * inv;
+    for (int k = ty; k < i; k += 16) {
+      const float vki = v[k * BASE_LD + i] * inv;
+      for (int c = i + ((tx - i) & 31); c < n; c += 32)
+        a[k * BASE_LD + c] = fmaf(-vki, a[i * BASE_LD + c], a[k * BASE_LD + c]);
     }
     __syncthreads();
-  }
-  for (int e = tid; e < n * n; e += BASE_THREADS) {
-    const int i = e / n, k = e % n;
-    Ublk[(long long)i * ld + k] = (i <= k) ? r[i * BASE_LD + k] : 0.f;
   }
 }
 

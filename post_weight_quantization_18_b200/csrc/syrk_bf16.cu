@@ -186,6 +186,7 @@ syrk_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_x,
         for (int c = 0; c < BN / 32; ++c) {
           const int col0 = jb * BN + c * 32;
           uint32_t r[32];
+          __syncwarp();  // tcgen05.ld is warp-collective: reconverge before every load
           const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) +
                                  (uint32_t)(buf * BN + c * 32);
           gptq::tmem_ld_32x32b_x32(taddr, r);

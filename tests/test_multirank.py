@@ -1,0 +1,59 @@
+"""Multi-rank host logic of bench.py on CPU: two gloo ranks, each with its own layer; only the
+timing crosses ranks (max over ranks)."""
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, q):
+    import sys
+    import datetime
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import torch.distributed as dist
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        got = bench.max_over_ranks([1.0 + rank, 10.0 - rank, 3.0], "cpu")
+        q.put((rank, got, bench.rank_seed_offset(rank)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_max_and_disjoint_seeds():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=5) for _ in range(2))
+    for rank, got, off in res:
+        assert got == [2.0, 10.0, 3.0]
+    assert res[0][2] != res[1][2]
+
+
+def test_single_process_identity():
+    import bench
+    assert bench.max_over_ranks([1.5, 2.5], "cpu") == [1.5, 2.5]
+
+
+def test_launch_accounting_matches_recursions():
+    """The bench's launch count follows the host recursions (d = 4096: 228 per step)."""
+    import bench
+    import layer_inputs as li
+    assert bench.launches_per_step(4096, li.WORKLOADS["llama7b_attn_proj"].quant) == 228
