@@ -186,15 +186,21 @@ GPTQ_DEV void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {
 GPTQ_DEV void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // Shared-memory matrix descriptor (tcgen05): start address, leading / stride byte offsets,
-// descriptor version 1, 128-byte swizzle.
-GPTQ_DEV uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+// descriptor version 1, layout type (2: 128-byte swizzle with 16-byte atoms; 1: 128-byte
+// swizzle with 32-byte atoms, the layout MN-major tf32 operands require).
+constexpr uint32_t kLayoutSW128 = 2, kLayoutSW128Atom32B = 1;
+GPTQ_DEV uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes,
+                            uint32_t layout) {
   uint64_t d = 0;
   d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
   d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
   d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
   d |= (uint64_t)1u << 46;  // version (sm_100)
-  d |= (uint64_t)2u << 61;  // SWIZZLE_128B
+  d |= (uint64_t)layout << 61;
   return d;
+}
+GPTQ_DEV uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  return smem_desc(saddr, lbo_bytes, sbo_bytes, kLayoutSW128);
 }
 
 // Instruction descriptor: fp32 accumulator, A/B format (1 = bf16, 2 = tf32), majorness

@@ -28,6 +28,11 @@ constexpr int SMEM_BYTES = SMEM_DATA + 1024 + 256;
 constexpr int THREADS = 320;
 constexpr int CONV_WARP0 = 2, N_CONV = 4, EPI_WARP0 = 6, N_EPI = 4;
 constexpr uint32_t TMEM_COLS = 256;                   // two 128 x 128 fp32 accumulators
+// The tensor core rounds toward zero when it adds into its fp32 accumulator, a one-sided error
+// of up to one ulp per accumulate step that grows linearly with K on sums of like-signed terms.
+// Each accumulator therefore covers at most KCB k-blocks (K = 1024, 384 accumulate steps);
+// consecutive chunks of a tile are folded into C in fp32 (round to nearest) by the epilogue.
+constexpr int KCB = 32;
 
 struct GemmArgs {
   int M, N, K;
@@ -42,12 +47,14 @@ struct GemmArgs {
 };
 
 // Shared-memory descriptor of one operand tile at K offset kk (in units of 8 elements).
-// K-major: rows of 128 B (32 fp32 of K) in 8-row swizzle atoms (SBO 1 KB); K steps move 32 B.
-// MN-major: four 32-element MN atoms of BK rows each (LBO 4 KB), 8-row K atoms (SBO 1 KB);
-// K steps move 8 rows = 1 KB.
+// K-major: rows of 128 B (32 fp32 of K), 128-byte swizzle with 16-byte atoms in 8-row groups
+// (SBO 1 KB); a K step moves 32 B along the row.
+// MN-major: tf32 operands stored MN-major must use the 128-byte swizzle with 32-byte atoms:
+// K rows of 128 B (32 fp32 of M or N) in 4-row groups (SBO 512 B), four 32-element MN atoms of
+// BK rows each (LBO 4 KB, one TMA box); a K step moves 8 rows = 1 KB.
 __device__ __forceinline__ uint64_t op_desc(uint32_t base, int mn_major, int kk) {
-  if (mn_major) return gptq::smem_desc_sw128(base + kk * 1024, 4096, 1024);
-  return gptq::smem_desc_sw128(base + kk * 32, 16, 1024);
+  if (mn_major) return gptq::smem_desc(base + kk * 1024, 4096, 512, gptq::kLayoutSW128Atom32B);
+  return gptq::smem_desc(base + kk * 32, 16, 1024, gptq::kLayoutSW128);
 }
 
 __device__ __forceinline__ void tile_of(int t, const GemmArgs& a, int& tm, int& tn) {
@@ -113,7 +120,7 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
           int tm, tn;
           tile_of(t, args, tm, tn);
           if (!tile_live(tm, tn, args)) continue;
-          for (int kb = 0; kb < nkb; ++kb) {
+          for (int kb = 0; kb < nkb; ++kb) {  // chunks of one tile are consecutive k-blocks
             if (!gptq::mbar_wait(&empty[stage], phase ^ 1, abort_flag)) break;
             uint8_t* sa = smem + stage * STAGE_BYTES;
             uint8_t* sb = sa + 2 * TILE_BYTES;
@@ -148,31 +155,35 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
           int tm, tn;
           tile_of(t, args, tm, tn);
           if (!tile_live(tm, tn, args)) continue;
-          if (!gptq::mbar_wait(&acc_empty[buf], acc_phase ^ 1, abort_flag)) break;
-          gptq::tc_fence_after();
-          const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
           bool ok = true;
-          for (int kb = 0; kb < nkb; ++kb) {
-            if (!gptq::mbar_wait(&conv[stage], phase, abort_flag)) { ok = false; break; }
+          for (int kc = 0; kc < nkb && ok; kc += KCB) {
+            const int kc1 = min(nkb, kc + KCB);
+            if (!gptq::mbar_wait(&acc_empty[buf], acc_phase ^ 1, abort_flag)) { ok = false; break; }
             gptq::tc_fence_after();
-            const uint32_t a_hi = gptq::smem_u32(smem + stage * STAGE_BYTES);
-            const uint32_t a_lo = a_hi + TILE_BYTES;
-            const uint32_t b_hi = a_hi + 2 * TILE_BYTES;
-            const uint32_t b_lo = a_hi + 3 * TILE_BYTES;
+            const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
+            for (int kb = kc; kb < kc1; ++kb) {
+              if (!gptq::mbar_wait(&conv[stage], phase, abort_flag)) { ok = false; break; }
+              gptq::tc_fence_after();
+              const uint32_t a_hi = gptq::smem_u32(smem + stage * STAGE_BYTES);
+              const uint32_t a_lo = a_hi + TILE_BYTES;
+              const uint32_t b_hi = a_hi + 2 * TILE_BYTES;
+              const uint32_t b_lo = a_hi + 3 * TILE_BYTES;
 #pragma unroll
-            for (int kk = 0; kk < BK / 8; ++kk) {
-              const uint64_t dah = op_desc(a_hi, args.a_mn, kk), dal = op_desc(a_lo, args.a_mn, kk);
-              const uint64_t dbh = op_desc(b_hi, args.b_mn, kk), dbl = op_desc(b_lo, args.b_mn, kk);
-              gptq::mma_tf32(d_tmem, dah, dbl, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
-              gptq::mma_tf32(d_tmem, dal, dbh, idesc, 1u);
-              gptq::mma_tf32(d_tmem, dah, dbh, idesc, 1u);
+              for (int kk = 0; kk < BK / 8; ++kk) {
+                const uint64_t dah = op_desc(a_hi, args.a_mn, kk), dal = op_desc(a_lo, args.a_mn, kk);
+                const uint64_t dbh = op_desc(b_hi, args.b_mn, kk), dbl = op_desc(b_lo, args.b_mn, kk);
+                gptq::mma_tf32(d_tmem, dah, dbl, idesc, (kb > kc || kk > 0) ? 1u : 0u);
+                gptq::mma_tf32(d_tmem, dal, dbh, idesc, 1u);
+                gptq::mma_tf32(d_tmem, dah, dbh, idesc, 1u);
+              }
+              gptq::mma_commit(&empty[stage]);
+              if (++stage == STAGES) { stage = 0; phase ^= 1; }
             }
-            gptq::mma_commit(&empty[stage]);
-            if (++stage == STAGES) { stage = 0; phase ^= 1; }
+            if (!ok) break;
+            gptq::mma_commit(&acc_full[buf]);
+            if (++buf == 2) { buf = 0; acc_phase ^= 1; }
           }
           if (!ok) break;
-          gptq::mma_commit(&acc_full[buf]);
-          if (++buf == 2) { buf = 0; acc_phase ^= 1; }
         }
       }
     } else if (warp < EPI_WARP0) {
@@ -218,7 +229,10 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
         int tm, tn;
         tile_of(t, args, tm, tn);
         if (!tile_live(tm, tn, args)) continue;
-        if (!gptq::mbar_wait(&acc_full[buf], acc_phase, abort_flag)) break;
+        bool ok = true;
+        for (int kc = 0; kc < nkb; kc += KCB) {
+        const float beta = (kc == 0) ? args.beta : 1.0f;  // later chunks fold into C
+        if (!gptq::mbar_wait(&acc_full[buf], acc_phase, abort_flag)) { ok = false; break; }
         gptq::tc_fence_after();
         const int row = tm * BM + quarter * 32 + lane;
 #pragma unroll 1
@@ -242,12 +256,12 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
                 o.y = args.alpha * __uint_as_float(r[4 * q + 1]);
                 o.z = args.alpha * __uint_as_float(r[4 * q + 2]);
                 o.w = args.alpha * __uint_as_float(r[4 * q + 3]);
-                if (args.beta != 0.f) {
+                if (beta != 0.f) {
                   const float4 old = *p;
-                  o.x = fmaf(args.beta, old.x, o.x);
-                  o.y = fmaf(args.beta, old.y, o.y);
-                  o.z = fmaf(args.beta, old.z, o.z);
-                  o.w = fmaf(args.beta, old.w, o.w);
+                  o.x = fmaf(beta, old.x, o.x);
+                  o.y = fmaf(beta, old.y, o.y);
+                  o.z = fmaf(beta, old.z, o.z);
+                  o.w = fmaf(beta, old.w, o.w);
                 }
                 *p = o;
               }
@@ -257,7 +271,7 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
                 const int col = col0 + e;
                 if (col >= args.N || (args.upper_only && row > col)) continue;
                 float o = args.alpha * __uint_as_float(r[e]);
-                if (args.beta != 0.f) o = fmaf(args.beta, crow[col], o);
+                if (beta != 0.f) o = fmaf(beta, crow[col], o);
                 crow[col] = o;
               }
             }
@@ -267,6 +281,8 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
         __syncwarp();
         if (lane == 0) gptq::mbar_arrive(&acc_empty[buf]);
         if (++buf == 2) { buf = 0; acc_phase ^= 1; }
+        }
+        if (!ok) break;
       }
     }
   }
@@ -296,15 +312,16 @@ int gemm_tf32x3(int M, int N, int K, float alpha, const float* A, long long lda,
                 bool upper_only, const int32_t* status, cudaStream_t stream) {
   CUtensorMap ta, tb;
   const CUtensorMapDataType f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
-  const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
+  const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;               // K-major tiles
+  const CUtensorMapSwizzle sw32 = CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B;    // MN-major tiles
   int rc;
   if (transA)  // MN-major: inner = M
-    rc = make_tmap_2d(&ta, f32, 4, A, (uint64_t)M, (uint64_t)K, (uint64_t)lda * 4, 32, BK, sw);
+    rc = make_tmap_2d(&ta, f32, 4, A, (uint64_t)M, (uint64_t)K, (uint64_t)lda * 4, 32, BK, sw32);
   else         // K-major: inner = K
     rc = make_tmap_2d(&ta, f32, 4, A, (uint64_t)K, (uint64_t)M, (uint64_t)lda * 4, BK, BM, sw);
   if (rc) return GPTQ_ERR_CUDA;
   if (!transB)  // MN-major: inner = N
-    rc = make_tmap_2d(&tb, f32, 4, B, (uint64_t)N, (uint64_t)K, (uint64_t)ldb * 4, 32, BK, sw);
+    rc = make_tmap_2d(&tb, f32, 4, B, (uint64_t)N, (uint64_t)K, (uint64_t)ldb * 4, 32, BK, sw32);
   else          // K-major: inner = K
     rc = make_tmap_2d(&tb, f32, 4, B, (uint64_t)K, (uint64_t)N, (uint64_t)ldb * 4, BK, BN, sw);
   if (rc) return GPTQ_ERR_CUDA;

@@ -119,64 +119,139 @@ __global__ void zero_lower_kernel(float* U, int d) {
   }
 }
 
-// Base block (n <= 128): H_d block (upper triangle, ld) -> U block = V^-1 where H_d = V V^T.
-// Phase 1 (Cholesky from the last column), step j: V_jj = sqrt(a_jj), V_ij = a_ij / V_jj, and the
-// leading block a_ik -= V_ij V_kj (i <= k < j). Phase 2 (U = V^-1, back substitution on all
-// columns at once), step i: row i of U = r_i / V_ii (written straight to global memory, it is
-// final) and r_kc -= V_ki U_ic for k < i, c >= i, starting from r = I. Every step reads only a
-// column (phase 1) or a row (phase 2) that the step itself does not write, so one barrier per
-// step suffices. Thread (ty, tx) of the 16 x 32 layout owns rows ty + 16a and columns = tx mod 32.
+// Base block (n <= 128): the damped block H_d (upper triangle, leading dimension ld) -> the
+// U block = V^-1 where H_d = V V^T, V upper. The same recursion as the host one, inside one CTA:
+//   128 -> 64 -> 32 on shared-memory matrices, with the four block products of every split
+//   done by all 16 warps, and 32 x 32 leaves factored and inverted by a single warp entirely in
+//   registers (lane = column; shuffles broadcast the pivot column, no block barriers).
+// A block smaller than 128 is padded at its end with the identity: the padded factor is block
+// diagonal, so the leading n x n part is unchanged.
 constexpr int BASE_THREADS = 512;
-constexpr int BASE_LD = gptq_host::kPrepBase + 1;
+constexpr int BN_ = gptq_host::kPrepBase;  // 128
+constexpr int BLD = BN_ + 1;               // padded leading dimension (conflict-free columns)
 
-__global__ void __launch_bounds__(BASE_THREADS)
-base_block_kernel(float* __restrict__ Hblk, float* __restrict__ Ublk, int n, int ld, int index0,
-                  int32_t* status) {
-  extern __shared__ float sm[];
-  float* a = sm;                                   // working matrix, then r
-  float* v = sm + gptq_host::kPrepBase * BASE_LD;  // V (upper)
-  __shared__ int bad;
-  const int tid = threadIdx.x, tx = tid & 31, ty = tid >> 5;
-  if (tid == 0) bad = gptq::status_bad(status) ? 1 : 0;
-  for (int i = ty; i < n; i += 16)
-    for (int k = tx; k < n; k += 32) a[i * BASE_LD + k] = (i <= k) ? Hblk[(long long)i * ld + k] : 0.f;
-  __syncthreads();
-  if (bad) return;
-  for (int j = n - 1; j >= 0; --j) {
-    const float piv = a[j * BASE_LD + j];
-    if (!(piv > 0.f) || !isfinite(piv)) {  // uniform: all threads read the same pivot
-      if (tid == 0) gptq::set_status(status, GPTQ_ERR_NOT_SPD, index0 + j);
-      return;
+// Leaf: A[o:o+32, o:o+32] (upper part) -> U[o:o+32, o:o+32] (upper, zeros below); one warp.
+// Returns false (uniformly) on a non-positive or non-finite pivot.
+__device__ bool leaf32(float* A, float* U, int o, int lane, int32_t* status, int index0) {
+  float a[32];  // column `lane` of the block: a[r] = A[o + r][o + lane] for r <= lane
+#pragma unroll
+  for (int r = 0; r < 32; ++r) a[r] = (r <= lane) ? A[(o + r) * BLD + o + lane] : 0.f;
+  bool ok = true;
+  // Cholesky from the last column: V_jj = sqrt(a_jj), V_rj = a_rj / V_jj, a_rl -= V_rj V_lj.
+#pragma unroll
+  for (int j = 31; j >= 0; --j) {
+    const float piv = __shfl_sync(0xffffffffu, a[j], j);
+    if (!(piv > 0.f) || !isfinite(piv)) {
+      ok = false;
+      if (lane == 0) gptq::set_status(status, GPTQ_ERR_NOT_SPD, index0 + o + j);
+      break;
     }
     const float vjj = sqrtf(piv);
     const float inv = 1.0f / vjj;
-    if (ty == 0) {
-      for (int i = tx; i < j; i += 32) v[i * BASE_LD + j] = a[i * BASE_LD + j] * inv;
-      if (tx == 0) v[j * BASE_LD + j] = vjj;
+    float vl = 0.f;
+#pragma unroll
+    for (int r = j - 1; r >= 0; --r) {
+      const float vr = __shfl_sync(0xffffffffu, a[r], j) * inv;  // V_rj from lane j
+      if (lane == r) vl = vr;
+      if (lane < j && r <= lane) a[r] = fmaf(-vr, vl, a[r]);
     }
-    for (int i = ty; i < j; i += 16) {
-      const float vij = a[i * BASE_LD + j] * inv;
-      for (int k = i + ((tx - i) & 31); k < j; k += 32)
-        a[i * BASE_LD + k] = fmaf(-vij, a[k * BASE_LD + j] * inv, a[i * BASE_LD + k]);
+    if (lane == j) {
+#pragma unroll
+      for (int r = 0; r < j; ++r) a[r] *= inv;
+      a[j] = vjj;
     }
-    __syncthreads();
   }
-  for (int i = ty; i < n; i += 16)
-    for (int k = tx; k < n; k += 32) {
-      a[i * BASE_LD + k] = (i == k) ? 1.f : 0.f;
-      if (k < i) Ublk[(long long)i * ld + k] = 0.f;
+  if (!ok) return false;
+  // U = V^-1: column `lane` by back substitution, V_rc fetched from lane c.
+  float u[32];
+#pragma unroll
+  for (int r = 0; r < 32; ++r) u[r] = 0.f;
+#pragma unroll
+  for (int r = 31; r >= 0; --r) {
+    const float vrr = __shfl_sync(0xffffffffu, a[r], r);
+    float sum = 0.f;
+#pragma unroll
+    for (int c = r + 1; c < 32; ++c) sum = fmaf(__shfl_sync(0xffffffffu, a[r], c), u[c], sum);
+    if (r == lane) u[r] = 1.0f / vrr;
+    else if (r < lane) u[r] = -sum / vrr;
+  }
+#pragma unroll
+  for (int r = 0; r < 32; ++r) U[(o + r) * BLD + o + lane] = u[r];
+  return true;
+}
+
+// C (m x m, smem) = alpha * op(X) op(Y) + beta * C, all operands m x m blocks in smem (ld BLD).
+// tx: 0 -> X[i][k], 1 -> X[k][i];  ty: 0 -> Y[k][n], 1 -> Y[n][k].
+template <int M>
+__device__ void block_gemm(float* C, const float* X, int tx, const float* Y, int ty, float alpha,
+                           float beta) {
+  for (int e = threadIdx.x; e < M * M; e += BASE_THREADS) {
+    const int i = e / M, n = e % M;
+    float acc = 0.f;
+#pragma unroll 8
+    for (int k = 0; k < M; ++k) {
+      const float x = tx ? X[k * BLD + i] : X[i * BLD + k];
+      const float y = ty ? Y[n * BLD + k] : Y[k * BLD + n];
+      acc = fmaf(x, y, acc);
     }
-  __syncthreads();
-  for (int i = n - 1; i >= 0; --i) {
-    const float inv = 1.0f / v[i * BASE_LD + i];
-    if (ty == 0)
-      for (int c = i + tx; c < n; c += 32) Ublk[(long long)i * ld + c] = a[i * BASE_LD + c] * inv;
-    for (int k = ty; k < i; k += 16) {
-      const float vki = v[k * BASE_LD + i] * inv;
-      for (int c = i + ((tx - i) & 31); c < n; c += 32)
-        a[k * BASE_LD + c] = fmaf(-vki, a[i * BASE_LD + c], a[k * BASE_LD + c]);
+    C[i * BLD + n] = (beta == 0.f) ? alpha * acc : fmaf(beta, C[i * BLD + n], alpha * acc);
+  }
+}
+
+template <int N>
+__device__ bool base_rec(float* A, float* U, int o, int32_t* status, int index0, int* fail) {
+  if constexpr (N == 32) {
+    if ((threadIdx.x >> 5) == 0) {
+      if (!leaf32(A, U, o, threadIdx.x & 31, status, index0) && (threadIdx.x & 31) == 0) *fail = 1;
     }
     __syncthreads();
+    return *fail == 0;
+  } else {
+    constexpr int m = N / 2;
+    float* Bb = A + o * BLD + o + m;          // A[o:o+m, o+m:o+N]
+    float* Aa = A + o * BLD + o;              // A[o:o+m, o:o+m]
+    float* U11 = U + o * BLD + o;
+    float* U12 = U + o * BLD + o + m;
+    float* U22 = U + (o + m) * BLD + o + m;
+    if (!base_rec<m>(A, U, o + m, status, index0, fail)) return false;
+    block_gemm<m>(U12, Bb, 0, U22, 1, 1.f, 0.f);     // T = B U22^T
+    __syncthreads();
+    block_gemm<m>(Aa, U12, 0, U12, 1, -1.f, 1.f);    // S = A - T T^T
+    __syncthreads();
+    if (!base_rec<m>(A, U, o, status, index0, fail)) return false;
+    block_gemm<m>(Bb, U12, 0, U22, 0, 1.f, 0.f);     // V = T U22
+    __syncthreads();
+    block_gemm<m>(U12, U11, 0, Bb, 0, -1.f, 0.f);    // U12 = -U11 V
+    __syncthreads();
+    return true;
+  }
+}
+
+__global__ void __launch_bounds__(BASE_THREADS)
+base_block_kernel(const float* __restrict__ Hblk, float* __restrict__ Ublk, int n, int ld,
+                  int index0, int32_t* status) {
+  extern __shared__ float sm[];
+  float* A = sm;
+  float* U = sm + BN_ * BLD;
+  __shared__ int bad, fail;
+  if (threadIdx.x == 0) {
+    bad = gptq::status_bad(status) ? 1 : 0;
+    fail = 0;
+  }
+  for (int e = threadIdx.x; e < BN_ * BN_; e += BASE_THREADS) {
+    const int i = e / BN_, k = e % BN_;
+    float v = 0.f;
+    if (i < n && k < n) v = (i <= k) ? Hblk[(long long)i * ld + k] : 0.f;
+    else if (i == k) v = 1.f;  // identity padding at the end
+    A[i * BLD + k] = v;
+    U[i * BLD + k] = 0.f;
+  }
+  __syncthreads();
+  if (bad) return;
+  if (!base_rec<BN_>(A, U, 0, status, index0, &fail)) return;
+  for (int e = threadIdx.x; e < n * n; e += BASE_THREADS) {
+    const int i = e / n, k = e % n;
+    Ublk[(long long)i * ld + k] = (i <= k) ? U[i * BLD + k] : 0.f;
   }
 }
 
@@ -223,7 +298,7 @@ int prep_zero_lower(float* U, int d, cudaStream_t stream) {
 
 int prep_base_block(float* Hblk, float* Ublk, int n, int ld, int index0, int32_t* status,
                     cudaStream_t stream) {
-  const size_t smem = 2 * (size_t)kPrepBase * BASE_LD * sizeof(float);
+  const size_t smem = 2 * (size_t)kPrepBase * BLD * sizeof(float);
   if (cudaFuncSetAttribute(base_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return GPTQ_ERR_CUDA;

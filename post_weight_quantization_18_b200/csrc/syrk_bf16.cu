@@ -273,21 +273,26 @@ int syrk_bf16_upper(float* H, int d, long long ldh, const void* X, long long n_t
   a.n_tiles = 0;
   for (int jb = 0; jb < a.n_jb; ++jb) a.n_tiles += (2 * jb + 2 < a.n_ib) ? 2 * jb + 2 : a.n_ib;
   a.nkb_total = (int)((n_tokens + BK - 1) / BK);
-  // Split the token range only as far as needed to fill the SMs: pick the split count
-  // (<= 64, every split non-empty) whose last wave is fullest, preferring >= 4 waves.
+  // The tensor core rounds toward zero when it adds into its fp32 accumulator (a one-sided
+  // error of up to one ulp per step on these like-signed sums), so one accumulator covers at
+  // most kMaxKb k-blocks (8192 tokens); the chunks are summed into H by the TMA reduce-add.
+  // Beyond that minimum, split the token range only as far as needed to fill the SMs: pick the
+  // split count whose last wave is fullest, preferring >= 4 waves.
+  constexpr int kMaxKb = 128;
   const int sms = num_sms();
-  int best_split = 1;
+  const int s_min = (a.nkb_total + kMaxKb - 1) / kMaxKb;
+  int best_split = s_min;
   double best_score = -1.0;
-  for (int s = 1; s <= 64 && s <= a.nkb_total; ++s) {
+  for (int s = s_min; s <= s_min + 64 && s <= a.nkb_total; ++s) {
     const int per = (a.nkb_total + s - 1) / s;
     const int s_eff = (a.nkb_total + per - 1) / per;
     if (s_eff != s) continue;
     const double units = (double)a.n_tiles * s;
     const double waves = units / sms;
     const double eff = waves / ceil(waves);
-    const double score = eff - (waves < 4.0 ? 0.25 : 0.0) - 0.002 * s;
+    const double score = eff - (waves < 4.0 ? 0.25 : 0.0) - 0.002 * (s - s_min);
     if (score > best_score) { best_score = score; best_split = s; }
-    if (a.n_tiles >= 8 * sms) break;  // plenty of tiles: no split
+    if ((double)a.n_tiles * s_min >= 8.0 * sms) break;  // plenty of units already
   }
   a.n_split = best_split;
   a.kb_per_split = (a.nkb_total + best_split - 1) / best_split;
