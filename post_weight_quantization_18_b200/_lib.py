@@ -55,7 +55,7 @@ def make_params(bits: int = 4, group_size: int = 128, sym: bool = False, order: 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is missing: build it with `python -m post_weight_quantization_18_b200.build`"
+            f"{LIB_PATH} is missing: build it with `python post_weight_quantization_18_b200/build.py`"
             " (there is no CPU fallback)")
     lib = ctypes.CDLL(LIB_PATH)
     P, I64, I32, F32, SZ = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float,

@@ -1,7 +1,9 @@
 """Build libgptq_b200.so in-tree with nvcc for sm_100a.
 
-    python -m post_weight_quantization_18_b200.build        # rebuild if sources changed
-    python -m post_weight_quantization_18_b200.build --force
+    python post_weight_quantization_18_b200/build.py          # rebuild if sources changed
+    python post_weight_quantization_18_b200/build.py --force
+
+(Run it as a script, not as `python -m`: importing the package loads the library.)
 
 Each .cu under csrc/ is compiled to an object (in parallel) and the objects are linked into one
 shared library next to this file. The CUDA runtime is linked statically; the driver API is
