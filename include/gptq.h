@@ -199,6 +199,33 @@ int rtn_quantize(const void* W, int w_dtype, int64_t ldw, int64_t d_out, int64_t
                  const gptq_params* p, uint8_t* codes, float* scales, float* zeros,
                  gptq_stream_t stream);
 
+/*
+ * gptq_quantize_layer_noalloc — gptq_quantize_layer for callers that cannot allocate device
+ * memory (for example a plugin running inside another runtime that owns all device memory, or a
+ * service that must not allocate once it is serving). It takes the same arguments minus
+ * (ws, ws_bytes) and produces the same outputs; the scratch comes from one fixed array of
+ * GPTQ_NOALLOC_SCRATCH_BYTES compiled into this library. (The source pages have no counterpart:
+ * this is an interface variant, not a step of the method.)
+ *
+ *   Limit: returns GPTQ_ERR_WORKSPACE, launching nothing, when
+ *          gptq_workspace_size(d_out, d_in, p) > GPTQ_NOALLOC_SCRATCH_BYTES (32 MiB: for example
+ *          4M weights such as 1024 x 4096 in natural order).
+ *   Memory: the array occupies GPTQ_NOALLOC_SCRATCH_BYTES of device memory on every GPU that
+ *          loads the library, until the process exits. The call itself allocates nothing.
+ *   Set-up: the first call on a device looks up the array's device address for that device
+ *          (cudaGetSymbolAddress, with the device current) and caches it; make that first call
+ *          before any stream capture.
+ *   Sharing: every call on a device uses the same array, and the array keeps the last call's
+ *          contents (nothing in it needs to start at zero). Calls whose kernels overlap on the GPU
+ *          (other streams, other host threads) race on the array: order them on one stream.
+ */
+#define GPTQ_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+int gptq_quantize_layer_noalloc(const void* W, int w_dtype, int64_t ldw, int64_t d_out,
+                                int64_t d_in, const float* U, const int32_t* perm,
+                                const uint8_t* dead, const gptq_params* p, uint8_t* codes,
+                                float* scales, float* zeros, int32_t* g_idx, int32_t* dev_status,
+                                gptq_stream_t stream);
+
 /* gptq_status_string — a static, human-readable name for a status code. */
 const char* gptq_status_string(int status);
 

@@ -31,7 +31,9 @@ GPTQ_ORDER_DESC_ACT = 1
 GPTQ_ORDER_GIVEN = 2
 
 EXPORTED = ("gptq_workspace_size", "gptq_hessian_accumulate", "gptq_prepare_hinv",
-            "gptq_quantize_layer", "gptq_pack", "rtn_quantize", "gptq_status_string")
+            "gptq_quantize_layer", "gptq_pack", "rtn_quantize", "gptq_status_string",
+            "gptq_quantize_layer_noalloc")
+GPTQ_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
 class GPTQError(RuntimeError):
@@ -69,6 +71,9 @@ def _load() -> ctypes.CDLL:
     lib.gptq_prepare_hinv.restype = I32
     lib.gptq_quantize_layer.argtypes = [P, I32, I64, I64, I64, P, P, P, PP, P, P, P, P, P, SZ, P, P]
     lib.gptq_quantize_layer.restype = I32
+    lib.gptq_quantize_layer_noalloc.argtypes = [P, I32, I64, I64, I64, P, P, P, PP, P, P, P, P,
+                                                P, P]
+    lib.gptq_quantize_layer_noalloc.restype = I32
     lib.gptq_pack.argtypes = [P, I64, I64, I32, P, P, I64, P, P, P, P]
     lib.gptq_pack.restype = I32
     lib.rtn_quantize.argtypes = [P, I32, I64, I64, I64, PP, P, P, P, P]
@@ -190,6 +195,36 @@ def gptq_quantize_layer(W: torch.Tensor, U: torch.Tensor, perm: torch.Tensor, de
                                   _ptr(zeros), _ptr(g_idx), _ptr(ws),
                                   ws.numel() * ws.element_size(), _ptr(dev_status), _stream())
     _check(rc, "gptq_quantize_layer")
+
+
+def gptq_quantize_layer_noalloc(W: torch.Tensor, U: torch.Tensor, perm: torch.Tensor,
+                                dead: torch.Tensor, params: gptq_params, codes: torch.Tensor,
+                                scales: torch.Tensor, zeros: torch.Tensor, g_idx: torch.Tensor,
+                                dev_status: torch.Tensor | None = None) -> None:
+    """gptq_quantize_layer with the library's own fixed scratch array instead of a caller buffer
+    (for callers that cannot allocate device memory); layers whose scratch exceeds
+    GPTQ_NOALLOC_SCRATCH_BYTES are rejected with GPTQ_ERR_WORKSPACE."""
+    _dev(W, "W", None, 2)
+    _row_major(W, "W")
+    n, d = W.shape
+    _dev(U, "U", torch.float32, 2)
+    _dev(codes, "codes", torch.uint8, 2)
+    _dev(scales, "scales", torch.float32, 2)
+    _dev(zeros, "zeros", torch.float32, 2)
+    _dev(g_idx, "g_idx", torch.int32, 1)
+    G = 1 if params.group_size == -1 else d // params.group_size
+    if codes.shape != (n, d) or not codes.is_contiguous():
+        raise ValueError("codes must be contiguous [d_out, d_in]")
+    if scales.shape != (n, G) or zeros.shape != (n, G) or not scales.is_contiguous() \
+            or not zeros.is_contiguous():
+        raise ValueError("scales / zeros must be contiguous [d_out, n_groups]")
+    if U.shape != (d, d) or g_idx.numel() != d:
+        raise ValueError("U must be d_in x d_in and g_idx must have d_in entries")
+    rc = _lib.gptq_quantize_layer_noalloc(_ptr(W), _dtype_code(W), W.stride(0), n, d, _ptr(U),
+                                          _ptr(perm), _ptr(dead), ctypes.byref(params),
+                                          _ptr(codes), _ptr(scales), _ptr(zeros), _ptr(g_idx),
+                                          _ptr(dev_status), _stream())
+    _check(rc, "gptq_quantize_layer_noalloc")
 
 
 def gptq_pack(codes: torch.Tensor, bits: int, scales: torch.Tensor, zeros: torch.Tensor,

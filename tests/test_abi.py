@@ -26,7 +26,8 @@ def declared_functions():
 def test_header_declares_the_boundary():
     assert declared_functions() == sorted([
         "gptq_hessian_accumulate", "gptq_pack", "gptq_prepare_hinv", "gptq_quantize_layer",
-        "gptq_status_string", "gptq_workspace_size", "rtn_quantize"])
+        "gptq_quantize_layer_noalloc", "gptq_status_string", "gptq_workspace_size",
+        "rtn_quantize"])
 
 
 def test_every_declared_symbol_is_exported(lib):
