@@ -130,79 +130,114 @@ constexpr int BASE_THREADS = 512;
 constexpr int BN_ = gptq_host::kPrepBase;  // 128
 constexpr int BLD = BN_ + 1;               // padded leading dimension (conflict-free columns)
 
-// Leaf: A[o:o+32, o:o+32] (upper part) -> U[o:o+32, o:o+32] (upper, zeros below); one warp.
-// Returns false (uniformly) on a non-positive or non-finite pivot.
-__device__ bool leaf32(float* A, float* U, int o, int lane, int32_t* status, int index0) {
-  float a[32];  // column `lane` of the block: a[r] = A[o + r][o + lane] for r <= lane
-#pragma unroll
-  for (int r = 0; r < 32; ++r) a[r] = (r <= lane) ? A[(o + r) * BLD + o + lane] : 0.f;
-  bool ok = true;
-  // Cholesky from the last column: V_jj = sqrt(a_jj), V_rj = a_rj / V_jj, a_rl -= V_rj V_lj.
-#pragma unroll
+// Leaf: A[o:o+32, o:o+32] (upper part) -> U[o:o+32, o:o+32] (upper, zeros below), computed by
+// warps 0-3 (128 threads) with a named barrier; V (32 x 33) is a separate shared array.
+//   Cholesky from the last column, step j: V_jj = sqrt(a_jj), V_rj = a_rj / V_jj (written to V),
+//   a_rk -= a_rj a_kj / a_jj for r <= k < j. A step reads column j of a and writes only columns
+//   < j of a and column j of V, so one barrier per step suffices.
+//   Inverse from U V = I, row by row: U_rc = (delta_rc - sum_{r<=k<c} U_rk V_kc) / V_cc; four
+//   threads share a row (partial sums over k = part mod 4, reduced with shuffles), rows are
+//   independent so no block barrier is needed.
+// Returns false (uniformly over the 128 threads) on a non-positive or non-finite pivot.
+constexpr int LEAF_THREADS = 128;
+constexpr int VLD = 33;
+
+__device__ __forceinline__ void leaf_bar() {
+  asm volatile("bar.sync 1, %0;" ::"n"(LEAF_THREADS) : "memory");
+}
+
+__device__ bool leaf32(float* A, float* U, float* V, int o, int t, int32_t* status, int index0) {
+  float* a = A + o * BLD + o;  // block view, ld BLD
+  const int lane = t & 31, w4 = t >> 5;  // warp w4 updates rows w4 + 4i, lane = column
   for (int j = 31; j >= 0; --j) {
-    const float piv = __shfl_sync(0xffffffffu, a[j], j);
+    const float piv = a[j * BLD + j];
     if (!(piv > 0.f) || !isfinite(piv)) {
-      ok = false;
-      if (lane == 0) gptq::set_status(status, GPTQ_ERR_NOT_SPD, index0 + o + j);
-      break;
+      if (t == 0) gptq::set_status(status, GPTQ_ERR_NOT_SPD, index0 + o + j);
+      return false;
     }
-    const float vjj = sqrtf(piv);
-    const float inv = 1.0f / vjj;
-    float vl = 0.f;
+    // The pivot's reciprocal square root from the special-function unit (about 1 ulp); the
+    // factor's own rounding in fp32 is of the same order.
+    const float inv = rsqrtf(piv);
+    if (w4 == 0) V[lane * VLD + j] = (lane < j) ? a[lane * BLD + j] * inv : (lane == j ? piv * inv : 0.f);
+    const float vk = a[lane * BLD + j] * inv;   // V_kj for k = lane
 #pragma unroll
-    for (int r = j - 1; r >= 0; --r) {
-      const float vr = __shfl_sync(0xffffffffu, a[r], j) * inv;  // V_rj from lane j
-      if (lane == r) vl = vr;
-      if (lane < j && r <= lane) a[r] = fmaf(-vr, vl, a[r]);
+    for (int i = 0; i < 8; ++i) {
+      const int r = w4 + 4 * i;
+      if (r <= lane && lane < j) a[r * BLD + lane] = fmaf(-a[r * BLD + j] * inv, vk, a[r * BLD + lane]);
     }
-    if (lane == j) {
-#pragma unroll
-      for (int r = 0; r < j; ++r) a[r] *= inv;
-      a[j] = vjj;
-    }
+    leaf_bar();
   }
-  if (!ok) return false;
-  // U = V^-1: column `lane` by back substitution, V_rc fetched from lane c.
-  float u[32];
-#pragma unroll
-  for (int r = 0; r < 32; ++r) u[r] = 0.f;
-#pragma unroll
-  for (int r = 31; r >= 0; --r) {
-    const float vrr = __shfl_sync(0xffffffffu, a[r], r);
-    float sum = 0.f;
-#pragma unroll
-    for (int c = r + 1; c < 32; ++c) sum = fmaf(__shfl_sync(0xffffffffu, a[r], c), u[c], sum);
-    if (r == lane) u[r] = 1.0f / vrr;
-    else if (r < lane) u[r] = -sum / vrr;
+  const int r = t >> 2, part = t & 3;
+  float* urow = U + (o + r) * BLD + o;
+  for (int c = 0; c < 32; ++c) {
+    float sp = 0.f;
+    for (int k = r + part; k < c; k += 4) sp = fmaf(urow[k], V[k * VLD + c], sp);
+    sp += __shfl_xor_sync(0xffffffffu, sp, 1);
+    sp += __shfl_xor_sync(0xffffffffu, sp, 2);
+    const float rc = __frcp_rn(V[c * VLD + c]);
+    const float uc = (c == r) ? rc : (c > r ? -sp * rc : 0.f);
+    if (part == 0) urow[c] = uc;
+    __syncwarp();
   }
-#pragma unroll
-  for (int r = 0; r < 32; ++r) U[(o + r) * BLD + o + lane] = u[r];
+  leaf_bar();
   return true;
 }
 
 // C (m x m, smem) = alpha * op(X) op(Y) + beta * C, all operands m x m blocks in smem (ld BLD).
 // tx: 0 -> X[i][k], 1 -> X[k][i];  ty: 0 -> Y[k][n], 1 -> Y[n][k].
+// m = 64: each thread owns rows {2r, 2r+1} and columns {c, c+16, c+32, c+48} (register tile).
 template <int M>
 __device__ void block_gemm(float* C, const float* X, int tx, const float* Y, int ty, float alpha,
                            float beta) {
-  for (int e = threadIdx.x; e < M * M; e += BASE_THREADS) {
-    const int i = e / M, n = e % M;
-    float acc = 0.f;
-#pragma unroll 8
+  if constexpr (M == 64) {
+    const int rb = threadIdx.x >> 4, cb = threadIdx.x & 15;
+    float acc[2][4] = {};
+#pragma unroll 4
     for (int k = 0; k < M; ++k) {
-      const float x = tx ? X[k * BLD + i] : X[i * BLD + k];
-      const float y = ty ? Y[n * BLD + k] : Y[k * BLD + n];
-      acc = fmaf(x, y, acc);
+      float x[2], y[4];
+#pragma unroll
+      for (int a = 0; a < 2; ++a) {
+        const int i = 2 * rb + a;
+        x[a] = tx ? X[k * BLD + i] : X[i * BLD + k];
+      }
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const int n = cb + 16 * b;
+        y[b] = ty ? Y[n * BLD + k] : Y[k * BLD + n];
+      }
+#pragma unroll
+      for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(x[a], y[b], acc[a][b]);
     }
-    C[i * BLD + n] = (beta == 0.f) ? alpha * acc : fmaf(beta, C[i * BLD + n], alpha * acc);
+#pragma unroll
+    for (int a = 0; a < 2; ++a)
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        float* cp = C + (2 * rb + a) * BLD + cb + 16 * b;
+        *cp = (beta == 0.f) ? alpha * acc[a][b] : fmaf(beta, *cp, alpha * acc[a][b]);
+      }
+  } else {
+    for (int e = threadIdx.x; e < M * M; e += BASE_THREADS) {
+      const int i = e / M, n = e % M;
+      float acc = 0.f;
+#pragma unroll 8
+      for (int k = 0; k < M; ++k) {
+        const float x = tx ? X[k * BLD + i] : X[i * BLD + k];
+        const float y = ty ? Y[n * BLD + k] : Y[k * BLD + n];
+        acc = fmaf(x, y, acc);
+      }
+      C[i * BLD + n] = (beta == 0.f) ? alpha * acc : fmaf(beta, C[i * BLD + n], alpha * acc);
+    }
   }
 }
 
 template <int N>
-__device__ bool base_rec(float* A, float* U, int o, int32_t* status, int index0, int* fail) {
+__device__ bool base_rec(float* A, float* U, float* V, int o, int32_t* status, int index0,
+                         int* fail) {
   if constexpr (N == 32) {
-    if ((threadIdx.x >> 5) == 0) {
-      if (!leaf32(A, U, o, threadIdx.x & 31, status, index0) && (threadIdx.x & 31) == 0) *fail = 1;
+    if (threadIdx.x < LEAF_THREADS) {
+      if (!leaf32(A, U, V, o, threadIdx.x, status, index0) && threadIdx.x == 0) *fail = 1;
     }
     __syncthreads();
     return *fail == 0;
@@ -213,12 +248,12 @@ __device__ bool base_rec(float* A, float* U, int o, int32_t* status, int index0,
     float* U11 = U + o * BLD + o;
     float* U12 = U + o * BLD + o + m;
     float* U22 = U + (o + m) * BLD + o + m;
-    if (!base_rec<m>(A, U, o + m, status, index0, fail)) return false;
+    if (!base_rec<m>(A, U, V, o + m, status, index0, fail)) return false;
     block_gemm<m>(U12, Bb, 0, U22, 1, 1.f, 0.f);     // T = B U22^T
     __syncthreads();
     block_gemm<m>(Aa, U12, 0, U12, 1, -1.f, 1.f);    // S = A - T T^T
     __syncthreads();
-    if (!base_rec<m>(A, U, o, status, index0, fail)) return false;
+    if (!base_rec<m>(A, U, V, o, status, index0, fail)) return false;
     block_gemm<m>(Bb, U12, 0, U22, 0, 1.f, 0.f);     // V = T U22
     __syncthreads();
     block_gemm<m>(U12, U11, 0, Bb, 0, -1.f, 0.f);    // U12 = -U11 V
@@ -233,6 +268,7 @@ base_block_kernel(const float* __restrict__ Hblk, float* __restrict__ Ublk, int 
   extern __shared__ float sm[];
   float* A = sm;
   float* U = sm + BN_ * BLD;
+  float* V = sm + 2 * BN_ * BLD;  // 32 x 33 leaf factor
   __shared__ int bad, fail;
   if (threadIdx.x == 0) {
     bad = gptq::status_bad(status) ? 1 : 0;
@@ -248,7 +284,7 @@ base_block_kernel(const float* __restrict__ Hblk, float* __restrict__ Ublk, int 
   }
   __syncthreads();
   if (bad) return;
-  if (!base_rec<BN_>(A, U, 0, status, index0, &fail)) return;
+  if (!base_rec<BN_>(A, U, V, 0, status, index0, &fail)) return;
   for (int e = threadIdx.x; e < n * n; e += BASE_THREADS) {
     const int i = e / n, k = e % n;
     Ublk[(long long)i * ld + k] = (i <= k) ? U[i * BLD + k] : 0.f;
@@ -298,7 +334,7 @@ int prep_zero_lower(float* U, int d, cudaStream_t stream) {
 
 int prep_base_block(float* Hblk, float* Ublk, int n, int ld, int index0, int32_t* status,
                     cudaStream_t stream) {
-  const size_t smem = 2 * (size_t)kPrepBase * BLD * sizeof(float);
+  const size_t smem = (2 * (size_t)kPrepBase * BLD + 32 * VLD) * sizeof(float);
   if (cudaFuncSetAttribute(base_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return GPTQ_ERR_CUDA;

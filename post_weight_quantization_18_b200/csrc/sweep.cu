@@ -12,10 +12,13 @@
 // current (compensated) values of its g columns; with one scale per row they come from the
 // row at the start of the sweep (sweep_row_params).
 //
-// Layout: one warp owns two rows (two independent dependency chains); lane l holds columns
-// 4l..4l+3 of each row in registers. Every lane evaluates the quantizer for column j on the
-// value broadcast from its owner lane, so no second broadcast is needed; the block's U
-// (128 x 128, zero below the diagonal) and 1/U_jj are staged in shared memory.
+// Layout: eight lanes own one row (four rows per warp); in each 32-column chunk of the block,
+// lane s of a row holds the four contiguous columns 4s..4s+3, so one row of U is read with
+// float4 loads, the remaining columns are spread evenly over the lanes, and chunks that are
+// already quantized are skipped uniformly. For column j the owner lane's value is broadcast
+// inside its 8-lane group, the group evaluates the quantizer, and the owner stores the code and
+// the error. The block's U (128 x 128, zero below the diagonal as gptq_prepare_hinv writes it)
+// arrives in shared memory with one TMA copy; 1/U_jj is computed from it.
 #include <float.h>
 
 #include <cuda_bf16.h>
@@ -26,10 +29,9 @@
 namespace {
 
 constexpr int BLK = 128;
-constexpr int SW_THREADS = 256;
-constexpr int RPW = 2;                                   // rows per warp
-constexpr int ROWS_PER_CTA = (SW_THREADS / 32) * RPW;    // 16
-constexpr int SW_SMEM = BLK * BLK * 4 + BLK * 4;
+constexpr int ROWS_PER_WARP = 4;
+constexpr int LANES_PER_ROW = 8;
+constexpr int SW_SMEM = BLK * BLK * 4 + BLK * 4 + 64;
 
 __device__ __forceinline__ float quant_code(float w, float s, float z, float maxq) {
   const float q = rintf(__fdiv_rn(w, s)) + z;
@@ -48,124 +50,130 @@ __device__ __forceinline__ void sym_params(float amax, int bits, float& s, float
   z = (float)(1 << (bits - 1));
 }
 
-__global__ void __launch_bounds__(SW_THREADS)
-sweep_block_kernel(const float* __restrict__ Wwork, const float* __restrict__ U,
+// Reductions over the eight lanes of a row group.
+__device__ __forceinline__ float group8_min(float v) {
+  v = fminf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+  v = fminf(v, __shfl_xor_sync(0xffffffffu, v, 2));
+  return fminf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+}
+__device__ __forceinline__ float group8_max(float v) {
+  v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+  v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
+  return fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+}
+
+__global__ void __launch_bounds__(128)
+sweep_block_kernel(const __grid_constant__ CUtensorMap tmap_u, const float* __restrict__ Wwork,
                    float* __restrict__ Err, uint8_t* __restrict__ codes,
                    float* __restrict__ scales, float* __restrict__ zeros, int n, int d, int col0,
                    int bits, int g, int sym, int32_t* status) {
-  extern __shared__ __align__(16) float sw_smem[];
-  float* Us = sw_smem;               // [128][128]
+  extern __shared__ __align__(128) float sw_smem[];
+  float* Us = sw_smem;                // [128][128], zero below the diagonal
   float* invd = sw_smem + BLK * BLK;  // [128]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(invd + BLK);
   __shared__ int bad;
+  __shared__ volatile int abort_flag;
   const int tid = threadIdx.x;
-  if (tid == 0) bad = gptq::status_bad(status) ? 1 : 0;
-  // Stage U[col0 .. col0+127][col0 .. col0+127] (entries below the diagonal forced to zero).
-  for (int e = tid; e < BLK * (BLK / 4); e += SW_THREADS) {
-    const int r = e / (BLK / 4), c4 = e % (BLK / 4);
-    float4 v = *reinterpret_cast<const float4*>(U + (long long)(col0 + r) * d + col0 + 4 * c4);
-    if (4 * c4 + 0 < r) v.x = 0.f;
-    if (4 * c4 + 1 < r) v.y = 0.f;
-    if (4 * c4 + 2 < r) v.z = 0.f;
-    if (4 * c4 + 3 < r) v.w = 0.f;
-    *reinterpret_cast<float4*>(Us + r * BLK + 4 * c4) = v;
+  if (tid == 0) {
+    bad = gptq::status_bad(status) ? 1 : 0;
+    abort_flag = 0;
+    gptq::mbar_init(bar, 1);
+    gptq::fence_barrier_init();
   }
-  if (tid < BLK) invd[tid] = __fdiv_rn(1.0f, U[(long long)(col0 + tid) * d + col0 + tid]);
   __syncthreads();
   if (bad) return;
-
+  if (tid == 0) {
+    gptq::mbar_arrive_expect_tx(bar, BLK * BLK * 4);
+    gptq::tma_load_2d(Us, &tmap_u, bar, col0, col0);
+  }
+  // Meanwhile: this thread's row of W.
   const int warp = tid >> 5, lane = tid & 31;
+  const int sub = lane & 7;                      // owns columns 32c + 4 sub + e
+  const int grp = lane & ~7;                     // first lane of this row's group
+  const int row = (blockIdx.x * (blockDim.x >> 5) + warp) * ROWS_PER_WARP + (lane >> 3);
+  const bool live = row < n;
+  const int rsafe = live ? row : 0;
   const float maxq = (float)((1 << bits) - 1);
   const int G = (g > 0) ? d / g : 1;
-  int row[RPW];
-  bool live[RPW];
-  float w[RPW][4], errv[RPW][4];
-  uint32_t cpack[RPW];
-  float s[RPW], z[RPW];
+  const float* wrow = Wwork + (long long)rsafe * d + col0 + 4 * sub;
+  float w[16];                                   // w[4c + e]: column 32c + 4 sub + e
 #pragma unroll
-  for (int rr = 0; rr < RPW; ++rr) {
-    row[rr] = blockIdx.x * ROWS_PER_CTA + warp * RPW + rr;
-    live[rr] = row[rr] < n;
-    const int rsafe = live[rr] ? row[rr] : 0;
-    const float4 v =
-        *reinterpret_cast<const float4*>(Wwork + (long long)rsafe * d + col0 + 4 * lane);
-    w[rr][0] = v.x; w[rr][1] = v.y; w[rr][2] = v.z; w[rr][3] = v.w;
-    cpack[rr] = 0u;
-    errv[rr][0] = errv[rr][1] = errv[rr][2] = errv[rr][3] = 0.f;
-    if (g <= 0) {  // one (s, z) per row, computed before the sweep
-      s[rr] = scales[rsafe];
-      z[rr] = zeros[rsafe];
-    } else {
-      s[rr] = 1.f;
-      z[rr] = 0.f;
-    }
+  for (int c = 0; c < 4; ++c) {
+    const float4 v = *reinterpret_cast<const float4*>(wrow + 32 * c);
+    w[4 * c + 0] = v.x; w[4 * c + 1] = v.y; w[4 * c + 2] = v.z; w[4 * c + 3] = v.w;
   }
-
-#pragma unroll 1
-  for (int l = 0; l < 32; ++l) {
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const int j = 4 * l + c;
-      if (g > 0 && (j % g) == 0) {
-        // Group [j, j+g): lanes j/4 .. (j+g)/4 - 1 hold its columns.
-        const bool in_grp = (4 * lane >= j) && (4 * lane < j + g);
-#pragma unroll
-        for (int rr = 0; rr < RPW; ++rr) {
-          float a, b;
-          if (sym) {
-            a = in_grp ? fmaxf(fmaxf(fabsf(w[rr][0]), fabsf(w[rr][1])),
-                               fmaxf(fabsf(w[rr][2]), fabsf(w[rr][3])))
-                       : 0.f;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-            sym_params(a, bits, s[rr], z[rr]);
-          } else {
-            a = in_grp ? fminf(fminf(w[rr][0], w[rr][1]), fminf(w[rr][2], w[rr][3])) : FLT_MAX;
-            b = in_grp ? fmaxf(fmaxf(w[rr][0], w[rr][1]), fmaxf(w[rr][2], w[rr][3])) : -FLT_MAX;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-              a = fminf(a, __shfl_xor_sync(0xffffffffu, a, o));
-              b = fmaxf(b, __shfl_xor_sync(0xffffffffu, b, o));
-            }
-            asym_params(a, b, maxq, s[rr], z[rr]);
-          }
-          if (lane == 0 && live[rr]) {
-            const long long gi = (long long)row[rr] * G + (col0 + j) / g;
-            scales[gi] = s[rr];
-            zeros[gi] = z[rr];
-          }
-        }
-      }
-      const float4 u4 = *reinterpret_cast<const float4*>(Us + j * BLK + 4 * lane);
-      const float id = invd[j];
-#pragma unroll
-      for (int rr = 0; rr < RPW; ++rr) {
-        const float wj = __shfl_sync(0xffffffffu, w[rr][c], l);
-        const float q = quant_code(wj, s[rr], z[rr], maxq);
-        const float wh = s[rr] * (q - z[rr]);
-        const float err = (wj - wh) * id;
-        if (lane == l) {
-          cpack[rr] |= ((uint32_t)q) << (8 * c);
-          errv[rr][c] = err;
-        }
-        w[rr][0] = fmaf(-err, u4.x, w[rr][0]);
-        w[rr][1] = fmaf(-err, u4.y, w[rr][1]);
-        w[rr][2] = fmaf(-err, u4.z, w[rr][2]);
-        w[rr][3] = fmaf(-err, u4.w, w[rr][3]);
-      }
-    }
+  float s = 1.f, z = 0.f;
+  if (g <= 0) {  // one (s, z) per row, computed before the sweep
+    s = scales[rsafe];
+    z = zeros[rsafe];
   }
+  const bool landed = gptq::mbar_wait(bar, 0, &abort_flag);
+  if (!__syncthreads_and(landed)) {  // the copy did not arrive in time: report, touch nothing
+    if (tid == 0) gptq::set_status(status, GPTQ_ERR_TIMEOUT, 3);
+    return;
+  }
+  for (int t = tid; t < BLK; t += blockDim.x) invd[t] = __fdiv_rn(1.0f, Us[t * BLK + t]);
+  __syncthreads();
 
+  float* erow = Err + (long long)rsafe * d + col0;
+  uint8_t* crow = codes + (long long)rsafe * d + col0;
   bool finite = true;
 #pragma unroll
-  for (int rr = 0; rr < RPW; ++rr) {
-    if (!live[rr]) continue;
-    *reinterpret_cast<uint32_t*>(codes + (long long)row[rr] * d + col0 + 4 * lane) = cpack[rr];
-    *reinterpret_cast<float4*>(Err + (long long)row[rr] * d + col0 + 4 * lane) =
-        make_float4(errv[rr][0], errv[rr][1], errv[rr][2], errv[rr][3]);
+  for (int c = 0; c < 4; ++c) {                  // 32-column chunks
+#pragma unroll 1
+    for (int so = 0; so < 8; ++so) {             // owner sub-lane within the chunk
 #pragma unroll
-    for (int c = 0; c < 4; ++c) finite = finite && (fabsf(errv[rr][c]) <= FLT_MAX);
+      for (int e = 0; e < 4; ++e) {
+        const int j = 32 * c + 4 * so + e;
+        if (g > 0 && (j % g) == 0) {
+          float a = sym ? 0.f : FLT_MAX, b = -FLT_MAX;
+#pragma unroll
+          for (int c2 = 0; c2 < 4; ++c2)
+#pragma unroll
+            for (int e2 = 0; e2 < 4; ++e2) {
+              const int k = 32 * c2 + 4 * sub + e2;
+              const float v = w[4 * c2 + e2];
+              if (k >= j && k < j + g) {
+                if (sym) a = fmaxf(a, fabsf(v));
+                else { a = fminf(a, v); b = fmaxf(b, v); }
+              }
+            }
+          if (sym) {
+            a = group8_max(a);
+            sym_params(a, bits, s, z);
+          } else {
+            a = group8_min(a);
+            b = group8_max(b);
+            asym_params(a, b, maxq, s, z);
+          }
+          if (sub == 0 && live) {
+            const long long gi = (long long)row * G + (col0 + j) / g;
+            scales[gi] = s;
+            zeros[gi] = z;
+          }
+        }
+        const float wj = __shfl_sync(0xffffffffu, w[4 * c + e], grp | so);
+        const float qv = quant_code(wj, s, z, maxq);
+        const float err = (wj - s * (qv - z)) * invd[j];
+        if (sub == so && live) {
+          crow[j] = (uint8_t)qv;
+          erow[j] = err;
+        }
+        finite = finite && (fabsf(err) <= FLT_MAX);
+        // w_k -= err * U_jk for the columns of chunks c..3 (U_jk = 0 for k < j).
+        const float* urow = Us + j * BLK + 4 * sub;
+#pragma unroll
+        for (int c2 = c; c2 < 4; ++c2) {
+          const float4 u = *reinterpret_cast<const float4*>(urow + 32 * c2);
+          w[4 * c2 + 0] = fmaf(-err, u.x, w[4 * c2 + 0]);
+          w[4 * c2 + 1] = fmaf(-err, u.y, w[4 * c2 + 1]);
+          w[4 * c2 + 2] = fmaf(-err, u.z, w[4 * c2 + 2]);
+          w[4 * c2 + 3] = fmaf(-err, u.w, w[4 * c2 + 3]);
+        }
+      }
+    }
   }
-  if (!finite) gptq::set_status(status, GPTQ_ERR_NONFINITE, col0);
+  if (!finite && live) gptq::set_status(status, GPTQ_ERR_NONFINITE, col0);
 }
 
 // Wwork[r][k] = dead[k] ? 0 : W[r][perm[k]] as fp32 (bf16 widened exactly).
@@ -274,10 +282,14 @@ int sweep_block(float* Wwork, const float* U, float* Err, uint8_t* codes, float*
   if (cudaFuncSetAttribute(sweep_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            SW_SMEM) != cudaSuccess)
     return GPTQ_ERR_CUDA;
-  const int grid = (n + ROWS_PER_CTA - 1) / ROWS_PER_CTA;
-  sweep_block_kernel<<<grid, SW_THREADS, SW_SMEM, stream>>>(Wwork, U, Err, codes, scales, zeros,
-                                                            n, d, col0, bits, group_size, sym,
-                                                            status);
+  CUtensorMap tu;  // the whole U (d x d fp32), copied 128 x 128 at a time without swizzle
+  if (make_tmap_2d(&tu, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, U, (uint64_t)d, (uint64_t)d,
+                   (uint64_t)d * 4, BLK, BLK, CU_TENSOR_MAP_SWIZZLE_NONE) != 0)
+    return GPTQ_ERR_CUDA;
+  const int warps_total = (n + ROWS_PER_WARP - 1) / ROWS_PER_WARP;
+  const int grid = (warps_total + 3) / 4;  // 4 warps (16 rows) per CTA
+  sweep_block_kernel<<<grid, 128, SW_SMEM, stream>>>(tu, Wwork, Err, codes, scales, zeros, n, d,
+                                                     col0, bits, group_size, sym, status);
   return cudaGetLastError() == cudaSuccess ? 0 : GPTQ_ERR_CUDA;
 }
 
