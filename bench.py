@@ -42,7 +42,13 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="calibration tokens instead of the workload's own count (smaller cases "
+                         "for profiler captures; the config line reports the count used)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--eager", action="store_true",
+                    help="call the C ABI directly in the timed steps instead of replaying the "
+                         "CUDA graphs recorded from the same calls")
     return ap.parse_args()
 
 
@@ -208,7 +214,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    wl = li.WORKLOADS[args.workload]
+    wl = workload(args)
     lin = wl.linears[0]
     act = wl.act(lin.act)
     tok_sample, row_sample = 4096, 32
@@ -247,6 +253,17 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def workload(args):
+    """The named workload, with its calibration token count replaced when --tokens is given."""
+    import dataclasses
+    import layer_inputs as li
+    wl = li.WORKLOADS[args.workload]
+    if args.tokens > 0:
+        acts = tuple(dataclasses.replace(a, n_tokens=args.tokens) for a in wl.acts)
+        wl = dataclasses.replace(wl, acts=acts)
+    return wl
+
+
 def config_dict(args, wl, world):
     lin = wl.linears[0]
     act = wl.act(lin.act)
@@ -257,7 +274,8 @@ def config_dict(args, wl, world):
                         f"damp={q.percdamp}{' act-order' if q.act_order else ''}",
             "d_out": lin.d_out, "d_in": lin.d_in, "n_tokens": act.n_tokens, "bits": q.bits,
             "group_size": q.group_size, "parallelism": f"{world} independent layer(s), one per GPU",
-            "l2": "inputs larger than L2 (X is 2 GiB) and a 256 MiB L2 flush between timed steps"}
+            "l2": f"X is {act.n_tokens * act.d * 2 / 2**30:.2f} GiB; a 256 MiB L2 flush between "
+                  "timed steps"}
 
 
 # ------------------------------------------------------------------------------------------
@@ -299,7 +317,7 @@ def run_ours(args):
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
 
-    wl = li.WORKLOADS[args.workload]
+    wl = workload(args)
     lin = wl.linears[0]
     act = wl.act(lin.act)
     q = wl.quant
@@ -335,23 +353,26 @@ def run_ours(args):
     outs_h = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (qweight, s16, z16, g_idx)]
 
     ev = {k: [] for k in ("step", "syrk", "prep", "quant", "pack")}
+    calls = [
+        lambda X, W: L.gptq_hessian_accumulate(H, X, 2.0, False, status),
+        lambda X, W: L.gptq_prepare_hinv(H, p, U, perm, dead, ws, status),
+        lambda X, W: L.gptq_quantize_layer(W, U, perm, dead, p, codes, scales, zeros, g_idx, ws,
+                                           status),
+        lambda X, W: L.gptq_pack(codes, q.bits, scales, zeros, qweight, s16, z16),
+    ]
 
-    def step(X, W, record):
+    def step(X, W, record, graphs=None):
         e = [torch.cuda.Event(enable_timing=True) for _ in range(5)] if record else None
         if record:
             e[0].record()
-        L.gptq_hessian_accumulate(H, X, 2.0, False, status)
+        for i, call in enumerate(calls):
+            if graphs is not None:
+                graphs[i].replay()
+            else:
+                call(X, W)
+            if record:
+                e[i + 1].record()
         if record:
-            e[1].record()
-        L.gptq_prepare_hinv(H, p, U, perm, dead, ws, status)
-        if record:
-            e[2].record()
-        L.gptq_quantize_layer(W, U, perm, dead, p, codes, scales, zeros, g_idx, ws, status)
-        if record:
-            e[3].record()
-        L.gptq_pack(codes, q.bits, scales, zeros, qweight, s16, z16)
-        if record:
-            e[4].record()
             ev["step"].append((e[0], e[4]))
             ev["syrk"].append((e[0], e[1]))
             ev["prep"].append((e[1], e[2]))
@@ -365,13 +386,28 @@ def run_ours(args):
     if st[0] != 0:
         raise RuntimeError(f"device status after warm-up: {G.status_string(st[0])} index {st[1]}")
 
+    # Record each C ABI call of the step once into a CUDA graph (the calls only enqueue
+    # kernels on the current stream) and replay the graphs in the timed steps: the ~230
+    # launches of a step then cost no host time and no launch gaps.
+    graphs = None
+    if not args.eager:
+        graphs = []
+        for call in calls:
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr):
+                call(Xd, Wd)
+            graphs.append(gr)
+        for gr in graphs:      # one untimed replay of the recorded step
+            gr.replay()
+        torch.cuda.synchronize()
+
     with ClockSampler(local) as clk:
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
         for _ in range(args.steps):
             flush.zero_()
-            step(Xd, Wd, True)
+            step(Xd, Wd, True, graphs)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
@@ -435,6 +471,8 @@ def run_ours(args):
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": statistics.mean(e2e_ms)},
             "gpu_launches": launches_per_step(d, q) * args.steps,
+            "execution": "eager C ABI calls" if args.eager else
+                         "CUDA graphs recorded from the C ABI calls, replayed",
             "clocks": clk.summary(),
             "cpu_baseline": cpu,
         }

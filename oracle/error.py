@@ -12,6 +12,8 @@ from __future__ import annotations
 
 import numpy as np
 
+from .hessian import as_f64
+
 
 def dequant_matrix(codes: np.ndarray, S: np.ndarray, Z: np.ndarray, g_idx: np.ndarray) -> np.ndarray:
     """W_hat [n, d] in original column order: s[g_idx[c]] * (code[c] - z[g_idx[c]])."""
@@ -44,6 +46,6 @@ def row_errors_direct(W_rows: np.ndarray, W_hat_rows: np.ndarray, X_tm: np.ndarr
     D = (np.asarray(W_rows, np.float64) - np.asarray(W_hat_rows, np.float64)).T   # [d, r]
     out = np.zeros(D.shape[1])
     for t0 in range(0, X_tm.shape[0], chunk):
-        y = np.asarray(X_tm[t0:t0 + chunk], np.float64) @ D
+        y = as_f64(X_tm[t0:t0 + chunk]) @ D
         out += np.sum(y * y, axis=0)
     return out

@@ -16,13 +16,19 @@ from __future__ import annotations
 import numpy as np
 
 
+def as_f64(x) -> np.ndarray:
+    """Exact float64 copy of a numpy array or of a CPU torch tensor (bf16 included)."""
+    if hasattr(x, "double") and hasattr(x, "numpy"):
+        return x.double().numpy()
+    return np.asarray(x, np.float64)
+
+
 def hessian(X_tm: np.ndarray, chunk: int = 16384) -> np.ndarray:
     """H = 2 X^T X over token-major X (float64), summed over token chunks with a library matmul."""
-    X_tm = np.asarray(X_tm)
     N, d = X_tm.shape
     H = np.zeros((d, d), np.float64)
     for t0 in range(0, N, chunk):
-        xc = np.asarray(X_tm[t0:t0 + chunk], np.float64)
+        xc = as_f64(X_tm[t0:t0 + chunk])
         H += xc.T @ xc
     return 2.0 * H
 
@@ -47,7 +53,7 @@ def hessian_rows(X_tm: np.ndarray, rows: np.ndarray, chunk: int = 16384) -> np.n
     rows = np.asarray(rows)
     out = np.zeros((rows.size, d), np.float64)
     for t0 in range(0, N, chunk):
-        xc = np.asarray(X_tm[t0:t0 + chunk], np.float64)
+        xc = as_f64(X_tm[t0:t0 + chunk])
         out += xc[:, rows].T @ xc
     return 2.0 * out
 
@@ -57,6 +63,6 @@ def hessian_diag(X_tm: np.ndarray, chunk: int = 16384) -> np.ndarray:
     N, d = X_tm.shape
     out = np.zeros(d, np.float64)
     for t0 in range(0, N, chunk):
-        xc = np.asarray(X_tm[t0:t0 + chunk], np.float64)
+        xc = as_f64(X_tm[t0:t0 + chunk])
         out += np.einsum("td,td->d", xc, xc)
     return 2.0 * out

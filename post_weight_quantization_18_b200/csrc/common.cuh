@@ -219,4 +219,7 @@ int make_tmap_2d(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, co
                  uint64_t inner, uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner,
                  uint32_t box_outer, CUtensorMapSwizzle swizzle);
 int num_sms();
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (kernel, device): later calls
+// make no runtime call, so the entry points can be recorded into a CUDA graph.
+int ensure_smem_attr(const void* func, int bytes);
 }  // namespace gptq_host

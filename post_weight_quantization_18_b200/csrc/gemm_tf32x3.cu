@@ -337,8 +337,7 @@ int gemm_tf32x3(int M, int N, int K, float alpha, const float* A, long long lda,
   a.n_tiles = a.tiles_m * a.tiles_n;
   a.status = status;
   a.status_w = const_cast<int32_t*>(status);
-  if (cudaFuncSetAttribute(gemm_tf32x3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           SMEM_BYTES) != cudaSuccess)
+  if (ensure_smem_attr(reinterpret_cast<const void*>(gemm_tf32x3_kernel), SMEM_BYTES) != 0)
     return GPTQ_ERR_CUDA;
   const int sms = num_sms();
   const int grid = a.n_tiles < sms ? a.n_tiles : sms;

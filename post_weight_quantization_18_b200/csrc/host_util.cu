@@ -1,6 +1,8 @@
 // host_util.cu — tensor-map encoding and device queries shared by the launchers.
 #include <cudaTypedefs.h>
 
+#include <mutex>
+
 #include "common.cuh"
 
 namespace gptq_host {
@@ -44,6 +46,22 @@ int num_sms() {
     n = 148;
   if (dev < 64) cached[dev] = n;
   return n;
+}
+
+int ensure_smem_attr(const void* func, int bytes) {
+  struct Entry { const void* f; int dev; int bytes; };
+  static Entry done[256];
+  static int n_done = 0;
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < n_done; ++i)
+    if (done[i].f == func && done[i].dev == dev && done[i].bytes >= bytes) return 0;
+  if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return -1;
+  if (n_done < 256) done[n_done++] = Entry{func, dev, bytes};
+  return 0;
 }
 
 }  // namespace gptq_host

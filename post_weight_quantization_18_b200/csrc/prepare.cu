@@ -130,56 +130,66 @@ constexpr int BASE_THREADS = 512;
 constexpr int BN_ = gptq_host::kPrepBase;  // 128
 constexpr int BLD = BN_ + 1;               // padded leading dimension (conflict-free columns)
 
-// Leaf: A[o:o+32, o:o+32] (upper part) -> U[o:o+32, o:o+32] (upper, zeros below), computed by
-// warps 0-3 (128 threads) with a named barrier; V (32 x 33) is a separate shared array.
-//   Cholesky from the last column, step j: V_jj = sqrt(a_jj), V_rj = a_rj / V_jj (written to V),
-//   a_rk -= a_rj a_kj / a_jj for r <= k < j. A step reads column j of a and writes only columns
-//   < j of a and column j of V, so one barrier per step suffices.
-//   Inverse from U V = I, row by row: U_rc = (delta_rc - sum_{r<=k<c} U_rk V_kc) / V_cc; four
-//   threads share a row (partial sums over k = part mod 4, reduced with shuffles), rows are
-//   independent so no block barrier is needed.
-// Returns false (uniformly over the 128 threads) on a non-positive or non-finite pivot.
-constexpr int LEAF_THREADS = 128;
+// Leaf: A[o:o+32, o:o+32] (upper part) -> U[o:o+32, o:o+32] (upper, zeros below); one warp,
+// lane r owns row r of the block in registers.
+//   Cholesky from the last column: at step s the pivot column j = 31 - s sits in a[31] (the
+//   registers rotate by one after every step, so the loop stays rolled with constant register
+//   indices). V_rj = a_rj / sqrt(a_jj) is computed by each lane for its own row and kept in the
+//   shared array V; then a_rk -= V_rj V_kj for r <= k < j with V_kj shuffled from lane k (the
+//   31 shuffles of a step are independent of each other).
+//   Inverse, row by row from U V = I: U_rc = (delta_rc - sum_{r<=k<c} U_rk V_kc) / V_cc, V read
+//   from shared memory (one broadcast per element).
+// Returns false (uniformly over the warp) on a non-positive or non-finite pivot.
 constexpr int VLD = 33;
 
-__device__ __forceinline__ void leaf_bar() {
-  asm volatile("bar.sync 1, %0;" ::"n"(LEAF_THREADS) : "memory");
-}
-
-__device__ bool leaf32(float* A, float* U, float* V, int o, int t, int32_t* status, int index0) {
-  float* a = A + o * BLD + o;  // block view, ld BLD
-  const int lane = t & 31, w4 = t >> 5;  // warp w4 updates rows w4 + 4i, lane = column
-  for (int j = 31; j >= 0; --j) {
-    const float piv = a[j * BLD + j];
+// One warp; N (16 or 32) rows, lanes >= N idle but present for the shuffles.
+template <int N>
+__device__ bool leaf(float* A, float* U, float* V, int o, int lane, int32_t* status,
+                     int index0) {
+  float a[N];
+#pragma unroll
+  for (int c = 0; c < N; ++c) a[c] = (lane < N && c >= lane) ? A[(o + lane) * BLD + o + c] : 0.f;
+#pragma unroll 1
+  for (int s = 0; s < N; ++s) {
+    const int j = N - 1 - s;
+    const float piv = __shfl_sync(0xffffffffu, a[N - 1], j);
     if (!(piv > 0.f) || !isfinite(piv)) {
-      if (t == 0) gptq::set_status(status, GPTQ_ERR_NOT_SPD, index0 + o + j);
+      if (lane == 0) gptq::set_status(status, GPTQ_ERR_NOT_SPD, index0 + o + j);
       return false;
     }
-    // The pivot's reciprocal square root from the special-function unit (about 1 ulp); the
-    // factor's own rounding in fp32 is of the same order.
+    // Reciprocal square root from the special-function unit (about 1 ulp, the order of the
+    // factor's own fp32 rounding).
     const float inv = rsqrtf(piv);
-    if (w4 == 0) V[lane * VLD + j] = (lane < j) ? a[lane * BLD + j] * inv : (lane == j ? piv * inv : 0.f);
-    const float vk = a[lane * BLD + j] * inv;   // V_kj for k = lane
+    const float v = (lane < j) ? a[N - 1] * inv : (lane == j ? piv * inv : 0.f);
+    if (lane < N) V[lane * VLD + j] = v;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int r = w4 + 4 * i;
-      if (r <= lane && lane < j) a[r * BLD + lane] = fmaf(-a[r * BLD + j] * inv, vk, a[r * BLD + lane]);
+    for (int idx = 0; idx < N - 1; ++idx) {
+      const int k = idx - s;  // column held in a[idx]
+      const float vk = __shfl_sync(0xffffffffu, v, k & 31);
+      if (k >= lane) a[idx] = fmaf(-v, vk, a[idx]);
     }
-    leaf_bar();
+#pragma unroll
+    for (int idx = N - 2; idx >= 0; --idx) a[idx + 1] = a[idx];
   }
-  const int r = t >> 2, part = t & 3;
-  float* urow = U + (o + r) * BLD + o;
-  for (int c = 0; c < 32; ++c) {
-    float sp = 0.f;
-    for (int k = r + part; k < c; k += 4) sp = fmaf(urow[k], V[k * VLD + c], sp);
-    sp += __shfl_xor_sync(0xffffffffu, sp, 1);
-    sp += __shfl_xor_sync(0xffffffffu, sp, 2);
-    const float rc = __frcp_rn(V[c * VLD + c]);
-    const float uc = (c == r) ? rc : (c > r ? -sp * rc : 0.f);
-    if (part == 0) urow[c] = uc;
-    __syncwarp();
+  __syncwarp();
+  if (lane < N) {
+    float u[N];
+#pragma unroll
+    for (int c = 0; c < N; ++c) {
+      float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+      for (int k = 0; k < c; ++k) {
+        const float t = u[k] * V[k * VLD + c];
+        if (k & 1) s1 += t;
+        else s0 += t;
+      }
+      const float rc = __frcp_rn(V[c * VLD + c]);
+      u[c] = (c == lane) ? rc : (c > lane ? -(s0 + s1) * rc : 0.f);
+    }
+#pragma unroll
+    for (int c = 0; c < N; ++c) U[(o + lane) * BLD + o + c] = u[c];
   }
-  leaf_bar();
+  __syncwarp();
   return true;
 }
 
@@ -232,12 +242,14 @@ __device__ void block_gemm(float* C, const float* X, int tx, const float* Y, int
   }
 }
 
+constexpr int kLeaf = 16;
+
 template <int N>
 __device__ bool base_rec(float* A, float* U, float* V, int o, int32_t* status, int index0,
                          int* fail) {
-  if constexpr (N == 32) {
-    if (threadIdx.x < LEAF_THREADS) {
-      if (!leaf32(A, U, V, o, threadIdx.x, status, index0) && threadIdx.x == 0) *fail = 1;
+  if constexpr (N == kLeaf) {
+    if (threadIdx.x < 32) {
+      if (!leaf<kLeaf>(A, U, V, o, threadIdx.x, status, index0) && threadIdx.x == 0) *fail = 1;
     }
     __syncthreads();
     return *fail == 0;
@@ -262,7 +274,7 @@ __device__ bool base_rec(float* A, float* U, float* V, int o, int32_t* status, i
   }
 }
 
-__global__ void __launch_bounds__(BASE_THREADS)
+__global__ void __launch_bounds__(BASE_THREADS, 1)
 base_block_kernel(const float* __restrict__ Hblk, float* __restrict__ Ublk, int n, int ld,
                   int index0, int32_t* status) {
   extern __shared__ float sm[];
@@ -335,8 +347,7 @@ int prep_zero_lower(float* U, int d, cudaStream_t stream) {
 int prep_base_block(float* Hblk, float* Ublk, int n, int ld, int index0, int32_t* status,
                     cudaStream_t stream) {
   const size_t smem = (2 * (size_t)kPrepBase * BLD + 32 * VLD) * sizeof(float);
-  if (cudaFuncSetAttribute(base_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem) != cudaSuccess)
+  if (ensure_smem_attr(reinterpret_cast<const void*>(base_block_kernel), (int)smem) != 0)
     return GPTQ_ERR_CUDA;
   base_block_kernel<<<1, BASE_THREADS, smem, stream>>>(Hblk, Ublk, n, ld, index0, status);
   return cudaGetLastError() == cudaSuccess ? 0 : GPTQ_ERR_CUDA;

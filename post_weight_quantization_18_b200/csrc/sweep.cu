@@ -279,8 +279,7 @@ int sweep_row_params(const float* Wwork, int n, int d, int bits, int sym, float*
 int sweep_block(float* Wwork, const float* U, float* Err, uint8_t* codes, float* scales,
                 float* zeros, int n, int d, int col0, int bits, int group_size, int sym,
                 int32_t* status, cudaStream_t stream) {
-  if (cudaFuncSetAttribute(sweep_block_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           SW_SMEM) != cudaSuccess)
+  if (ensure_smem_attr(reinterpret_cast<const void*>(sweep_block_kernel), SW_SMEM) != 0)
     return GPTQ_ERR_CUDA;
   CUtensorMap tu;  // the whole U (d x d fp32), copied 128 x 128 at a time without swizzle
   if (make_tmap_2d(&tu, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, U, (uint64_t)d, (uint64_t)d,

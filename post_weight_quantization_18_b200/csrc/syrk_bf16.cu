@@ -300,8 +300,7 @@ int syrk_bf16_upper(float* H, int d, long long ldh, const void* X, long long n_t
   a.alpha = alpha;
   a.status = status;
 
-  if (cudaFuncSetAttribute(syrk_bf16_tcgen05_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           SMEM_BYTES) != cudaSuccess)
+  if (ensure_smem_attr(reinterpret_cast<const void*>(syrk_bf16_tcgen05_kernel), SMEM_BYTES) != 0)
     return GPTQ_ERR_CUDA;
   const int grid = (int)(a.n_units < sms ? a.n_units : sms);
   syrk_bf16_tcgen05_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tx, th, a);
