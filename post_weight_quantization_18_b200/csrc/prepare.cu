@@ -120,155 +120,176 @@ __global__ void zero_lower_kernel(float* U, int d) {
 }
 
 // Base block (n <= 128): the damped block H_d (upper triangle, leading dimension ld) -> the
-// U block = V^-1 where H_d = V V^T, V upper. The same recursion as the host one, inside one CTA:
-//   128 -> 64 -> 32 on shared-memory matrices, with the four block products of every split
-//   done by all 16 warps, and 32 x 32 leaves factored and inverted by a single warp entirely in
-//   registers (lane = column; shuffles broadcast the pivot column, no block barriers).
+// U block = V^-1 where H_d = V V^T, V upper. The same recursion as the host one, inside one CTA
+// of 16 warps on two shared-memory matrices (A: the block being factored, U: the result):
+//   128 -> 64 -> 32 -> 16-column leaves. Each split does the four block products of the host
+//   recursion on the tensor cores (warp-level m16n8k8 TF32 with the three-term hi/lo split, so
+//   the products carry fp32 accuracy), skipping the k-ranges where the triangular operand is
+//   zero and computing only the upper tiles of the symmetric update. A leaf is factored and
+//   inverted by one warp in registers (no block barriers inside).
 // A block smaller than 128 is padded at its end with the identity: the padded factor is block
 // diagonal, so the leading n x n part is unchanged.
 constexpr int BASE_THREADS = 512;
+constexpr int BASE_WARPS = BASE_THREADS / 32;
 constexpr int BN_ = gptq_host::kPrepBase;  // 128
-constexpr int BLD = BN_ + 1;               // padded leading dimension (conflict-free columns)
+// Row pitch of the shared-memory matrices. 132 = 4 (mod 32) puts rows g = 0..7 of a fragment
+// on banks 4g, so the 8 rows x 4 columns that an m16n8k8 operand fragment reads hit 32
+// distinct banks; rows stay 16-byte aligned for vector copies.
+constexpr int BLD = BN_ + 4;
+constexpr int U_OFF = BN_ * BLD;           // U follows A in shared memory
+constexpr int kLeaf = 16;
 
-// Leaf: A[o:o+32, o:o+32] (upper part) -> U[o:o+32, o:o+32] (upper, zeros below); one warp,
-// lane r owns row r of the block in registers.
-//   Cholesky from the last column: at step s the pivot column j = 31 - s sits in a[31] (the
-//   registers rotate by one after every step, so the loop stays rolled with constant register
-//   indices). V_rj = a_rj / sqrt(a_jj) is computed by each lane for its own row and kept in the
-//   shared array V; then a_rk -= V_rj V_kj for r <= k < j with V_kj shuffled from lane k (the
-//   31 shuffles of a step are independent of each other).
-//   Inverse, row by row from U V = I: U_rc = (delta_rc - sum_{r<=k<c} U_rk V_kc) / V_cc, V read
-//   from shared memory (one broadcast per element).
-// Returns false (uniformly over the warp) on a non-positive or non-finite pivot.
-constexpr int VLD = 33;
-
-// One warp; N (16 or 32) rows, lanes >= N idle but present for the shuffles.
-template <int N>
-__device__ bool leaf(float* A, float* U, float* V, int o, int lane, int32_t* status,
-                     int index0) {
-  float a[N];
+// Leaf: A[o:o+16, o:o+16] (upper part) -> U[o:o+16, o:o+16] (upper, zeros below). One warp.
+//   Cholesky from the last column, lane r owning row r: at step j the pivot a_jj arrives by
+//   shuffle, V_rj = a_rj / sqrt(a_jj) is formed by each lane for its own row and kept in
+//   registers (vrow), and a_rk -= V_rj V_kj for r <= k < j with V_kj shuffled from lane k.
+//   Inverse by back substitution with lane c owning column c of U (U V = I read column-wise:
+//   V U = I): U_cc = 1/V_cc = rsqrt(a_cc) and, for r < c, U_rc = -(sum_{r<k<=c} V_rk U_kc)/V_rr
+//   with V_rk shuffled from lane r; the newest term enters each sum last.
+// Returns -1, or the first leaf column (in factorization order) whose pivot is not positive
+// and finite; the value is the same on every lane.
+__device__ __noinline__ int leaf16(int o) {
+  extern __shared__ float sm[];
+  const int lane = threadIdx.x & 31;
+  constexpr int N = kLeaf;
+  float a[N], vrow[N], rinv[N];
 #pragma unroll
-  for (int c = 0; c < N; ++c) a[c] = (lane < N && c >= lane) ? A[(o + lane) * BLD + o + c] : 0.f;
-#pragma unroll 1
-  for (int s = 0; s < N; ++s) {
-    const int j = N - 1 - s;
-    const float piv = __shfl_sync(0xffffffffu, a[N - 1], j);
-    if (!(piv > 0.f) || !isfinite(piv)) {
-      if (lane == 0) gptq::set_status(status, GPTQ_ERR_NOT_SPD, index0 + o + j);
-      return false;
-    }
+  for (int c = 0; c < N; ++c) a[c] = (lane < N && c >= lane) ? sm[(o + lane) * BLD + o + c] : 0.f;
+  int badj = -1;
+#pragma unroll
+  for (int j = N - 1; j >= 0; --j) {
+    const float piv = __shfl_sync(0xffffffffu, a[j], j);
+    if (badj < 0 && !(piv > 0.f && piv <= 3.402823466e38f)) badj = j;
     // Reciprocal square root from the special-function unit (about 1 ulp, the order of the
     // factor's own fp32 rounding).
     const float inv = rsqrtf(piv);
-    const float v = (lane < j) ? a[N - 1] * inv : (lane == j ? piv * inv : 0.f);
-    if (lane < N) V[lane * VLD + j] = v;
+    rinv[j] = inv;
+    const float v = (lane < j) ? a[j] * inv : (lane == j ? piv * inv : 0.f);
+    vrow[j] = v;
 #pragma unroll
-    for (int idx = 0; idx < N - 1; ++idx) {
-      const int k = idx - s;  // column held in a[idx]
-      const float vk = __shfl_sync(0xffffffffu, v, k & 31);
-      if (k >= lane) a[idx] = fmaf(-v, vk, a[idx]);
+    for (int k = 0; k < j; ++k) {
+      const float vk = __shfl_sync(0xffffffffu, v, k);
+      if (k >= lane) a[k] = fmaf(-v, vk, a[k]);
     }
-#pragma unroll
-    for (int idx = N - 2; idx >= 0; --idx) a[idx + 1] = a[idx];
   }
-  __syncwarp();
+  float u[N];
+#pragma unroll
+  for (int r = N - 1; r >= 0; --r) {
+    float s = 0.f;
+#pragma unroll
+    for (int k = N - 1; k > r; --k) s = fmaf(__shfl_sync(0xffffffffu, vrow[k], r), u[k], s);
+    u[r] = (r == lane) ? rinv[r] : (r < lane ? -s * rinv[r] : 0.f);
+  }
   if (lane < N) {
-    float u[N];
 #pragma unroll
-    for (int c = 0; c < N; ++c) {
-      float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-      for (int k = 0; k < c; ++k) {
-        const float t = u[k] * V[k * VLD + c];
-        if (k & 1) s1 += t;
-        else s0 += t;
-      }
-      const float rc = __frcp_rn(V[c * VLD + c]);
-      u[c] = (c == lane) ? rc : (c > lane ? -(s0 + s1) * rc : 0.f);
-    }
-#pragma unroll
-    for (int c = 0; c < N; ++c) U[(o + lane) * BLD + o + c] = u[c];
+    for (int k = 0; k < N; ++k) sm[U_OFF + (o + k) * BLD + o + lane] = u[k];
   }
   __syncwarp();
-  return true;
+  return badj;
 }
 
-// C (m x m, smem) = alpha * op(X) op(Y) + beta * C, all operands m x m blocks in smem (ld BLD).
-// tx: 0 -> X[i][k], 1 -> X[k][i];  ty: 0 -> Y[k][n], 1 -> Y[n][k].
-// m = 64: each thread owns rows {2r, 2r+1} and columns {c, c+16, c+32, c+48} (register tile).
-template <int M>
-__device__ void block_gemm(float* C, const float* X, int tx, const float* Y, int ty, float alpha,
-                           float beta) {
-  if constexpr (M == 64) {
-    const int rb = threadIdx.x >> 4, cb = threadIdx.x & 15;
-    float acc[2][4] = {};
-#pragma unroll 4
-    for (int k = 0; k < M; ++k) {
-      float x[2], y[4];
+// Which operand of a block product is triangular, so that whole k-steps can be skipped, or
+// whether only the upper output tiles are wanted.
+enum : int {
+  kFull = 0,
+  kYUpperTransposed = 1,  // Y[n][k] upper (read transposed): terms with k < n vanish
+  kCUpperOnly = 2,        // symmetric result: output tiles below the diagonal are not needed
+  kYUpper = 3,            // Y[k][n] upper: terms with k > n vanish
+  kXUpper = 4,            // X[i][k] upper: terms with k < i vanish
+};
+
+GPTQ_DEV uint32_t tf32_hi(float x) { return __float_as_uint(x) & 0xffffe000u; }
+GPTQ_DEV uint32_t tf32_lo(float x, uint32_t hi) { return __float_as_uint(x - __uint_as_float(hi)); }
+
+GPTQ_DEV void mma_m16n8k8_tf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// C (m x m) = alpha * X Y' + beta * C on shared-memory blocks (offsets into the dynamic shared
+// array, pitch BLD), Y' = Y (ty = 0, Y[k][n]) or Y^T (ty = 1, Y[n][k]). Warps w0 .. w0+nw-1
+// take 16 x 16 output tiles in turn. Each product x*y is formed as
+// hi(x)hi(y) + hi(x)lo(y) + lo(x)hi(y) with hi the operand's top 19 bits (TF32) and lo the rest.
+__device__ __noinline__ void block_mma(int m, int c_off, int x_off, int y_off, int ty,
+                                       float alpha, float beta, int tri, int w0, int nw) {
+  extern __shared__ float sm[];
+  const int warp = (threadIdx.x >> 5) - w0, lane = threadIdx.x & 31;
+  if (warp < 0 || warp >= nw) return;
+  const int g = lane >> 2, t = lane & 3;
+  const int tiles = m >> 4;
+  const float* X = sm + x_off;
+  const float* Y = sm + y_off;
+  float* C = sm + c_off;
+  for (int tile = warp; tile < tiles * tiles; tile += nw) {
+    const int i0 = (tile / tiles) * 16, n0 = (tile % tiles) * 16;
+    if (tri == kCUpperOnly && i0 > n0) continue;
+    int k_lo = 0, k_hi = m;
+    if (tri == kYUpperTransposed) k_lo = n0;
+    if (tri == kYUpper) k_hi = n0 + 16;
+    if (tri == kXUpper) k_lo = i0;
+    float hh[2][4] = {}, cross[2][4] = {};
+    for (int k0 = k_lo; k0 < k_hi; k0 += 8) {
+      const float xa[4] = {X[(i0 + g) * BLD + k0 + t], X[(i0 + g + 8) * BLD + k0 + t],
+                           X[(i0 + g) * BLD + k0 + t + 4], X[(i0 + g + 8) * BLD + k0 + t + 4]};
+      uint32_t ah[4], al[4];
 #pragma unroll
-      for (int a = 0; a < 2; ++a) {
-        const int i = 2 * rb + a;
-        x[a] = tx ? X[k * BLD + i] : X[i * BLD + k];
+      for (int q = 0; q < 4; ++q) {
+        ah[q] = tf32_hi(xa[q]);
+        al[q] = tf32_lo(xa[q], ah[q]);
       }
 #pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        const int n = cb + 16 * b;
-        y[b] = ty ? Y[n * BLD + k] : Y[k * BLD + n];
+      for (int h = 0; h < 2; ++h) {
+        const int n = n0 + 8 * h + g;
+        const float y0 = ty ? Y[n * BLD + k0 + t] : Y[(k0 + t) * BLD + n];
+        const float y1 = ty ? Y[n * BLD + k0 + t + 4] : Y[(k0 + t + 4) * BLD + n];
+        const uint32_t bh0 = tf32_hi(y0), bh1 = tf32_hi(y1);
+        mma_m16n8k8_tf32(cross[h], ah, tf32_lo(y0, bh0), tf32_lo(y1, bh1));
+        mma_m16n8k8_tf32(cross[h], al, bh0, bh1);
+        mma_m16n8k8_tf32(hh[h], ah, bh0, bh1);
       }
-#pragma unroll
-      for (int a = 0; a < 2; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = fmaf(x[a], y[b], acc[a][b]);
     }
 #pragma unroll
-    for (int a = 0; a < 2; ++a)
+    for (int h = 0; h < 2; ++h)
 #pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        float* cp = C + (2 * rb + a) * BLD + cb + 16 * b;
-        *cp = (beta == 0.f) ? alpha * acc[a][b] : fmaf(beta, *cp, alpha * acc[a][b]);
+      for (int q = 0; q < 4; ++q) {
+        float* cp = C + (i0 + g + ((q & 2) ? 8 : 0)) * BLD + n0 + 8 * h + 2 * t + (q & 1);
+        const float v = alpha * (hh[h][q] + cross[h][q]);
+        *cp = (beta == 0.f) ? v : fmaf(beta, *cp, v);
       }
-  } else {
-    for (int e = threadIdx.x; e < M * M; e += BASE_THREADS) {
-      const int i = e / M, n = e % M;
-      float acc = 0.f;
-#pragma unroll 8
-      for (int k = 0; k < M; ++k) {
-        const float x = tx ? X[k * BLD + i] : X[i * BLD + k];
-        const float y = ty ? Y[n * BLD + k] : Y[k * BLD + n];
-        acc = fmaf(x, y, acc);
-      }
-      C[i * BLD + n] = (beta == 0.f) ? alpha * acc : fmaf(beta, C[i * BLD + n], alpha * acc);
-    }
   }
 }
-
-constexpr int kLeaf = 16;
 
 template <int N>
-__device__ bool base_rec(float* A, float* U, float* V, int o, int32_t* status, int index0,
-                         int* fail) {
+__device__ __forceinline__ bool base_rec(int o, int32_t* status, int index0, int* fail) {
   if constexpr (N == kLeaf) {
     if (threadIdx.x < 32) {
-      if (!leaf<kLeaf>(A, U, V, o, threadIdx.x, status, index0) && threadIdx.x == 0) *fail = 1;
+      const int badj = leaf16(o);
+      if (badj >= 0 && threadIdx.x == 0) {
+        gptq::set_status(status, GPTQ_ERR_NOT_SPD, index0 + o + badj);
+        *fail = 1;
+      }
     }
     __syncthreads();
     return *fail == 0;
   } else {
     constexpr int m = N / 2;
-    float* Bb = A + o * BLD + o + m;          // A[o:o+m, o+m:o+N]
-    float* Aa = A + o * BLD + o;              // A[o:o+m, o:o+m]
-    float* U11 = U + o * BLD + o;
-    float* U12 = U + o * BLD + o + m;
-    float* U22 = U + (o + m) * BLD + o + m;
-    if (!base_rec<m>(A, U, V, o + m, status, index0, fail)) return false;
-    block_gemm<m>(U12, Bb, 0, U22, 1, 1.f, 0.f);     // T = B U22^T
+    const int Bb = o * BLD + o + m;             // A[o:o+m, o+m:o+N]
+    const int Aa = o * BLD + o;                 // A[o:o+m, o:o+m]
+    const int U11 = U_OFF + o * BLD + o;
+    const int U12 = U_OFF + o * BLD + o + m;
+    const int U22 = U_OFF + (o + m) * BLD + o + m;
+    if (!base_rec<m>(o + m, status, index0, fail)) return false;
+    block_mma(m, U12, Bb, U22, 1, 1.f, 0.f, kYUpperTransposed, 0, BASE_WARPS);  // T = B U22^T
     __syncthreads();
-    block_gemm<m>(Aa, U12, 0, U12, 1, -1.f, 1.f);    // S = A - T T^T
+    // S = A - T T^T (upper tiles) and V = T U22 both need only T: one barrier for the two.
+    block_mma(m, Aa, U12, U12, 1, -1.f, 1.f, kCUpperOnly, 0, BASE_WARPS / 2);
+    block_mma(m, Bb, U12, U22, 0, 1.f, 0.f, kYUpper, BASE_WARPS / 2, BASE_WARPS / 2);
     __syncthreads();
-    if (!base_rec<m>(A, U, V, o, status, index0, fail)) return false;
-    block_gemm<m>(Bb, U12, 0, U22, 0, 1.f, 0.f);     // V = T U22
-    __syncthreads();
-    block_gemm<m>(U12, U11, 0, Bb, 0, -1.f, 0.f);    // U12 = -U11 V
+    if (!base_rec<m>(o, status, index0, fail)) return false;
+    block_mma(m, U12, U11, Bb, 0, -1.f, 0.f, kXUpper, 0, BASE_WARPS);          // U12 = -U11 V
     __syncthreads();
     return true;
   }
@@ -278,28 +299,60 @@ __global__ void __launch_bounds__(BASE_THREADS, 1)
 base_block_kernel(const float* __restrict__ Hblk, float* __restrict__ Ublk, int n, int ld,
                   int index0, int32_t* status) {
   extern __shared__ float sm[];
-  float* A = sm;
-  float* U = sm + BN_ * BLD;
-  float* V = sm + 2 * BN_ * BLD;  // 32 x 33 leaf factor
   __shared__ int bad, fail;
   if (threadIdx.x == 0) {
     bad = gptq::status_bad(status) ? 1 : 0;
     fail = 0;
   }
-  for (int e = threadIdx.x; e < BN_ * BN_; e += BASE_THREADS) {
-    const int i = e / BN_, k = e % BN_;
-    float v = 0.f;
-    if (i < n && k < n) v = (i <= k) ? Hblk[(long long)i * ld + k] : 0.f;
-    else if (i == k) v = 1.f;  // identity padding at the end
-    A[i * BLD + k] = v;
-    U[i * BLD + k] = 0.f;
+  const bool vec = (n == BN_) && (ld % 4 == 0) && ((reinterpret_cast<uintptr_t>(Hblk) & 15) == 0) &&
+                   ((reinterpret_cast<uintptr_t>(Ublk) & 15) == 0);
+  if (vec) {
+    // Full block: all eight 16-byte loads of a thread are issued before any is used.
+    constexpr int kPer = BN_ * BN_ / 4 / BASE_THREADS;  // 8
+    float4 v[kPer];
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+      const int e = (q * BASE_THREADS + threadIdx.x) * 4, i = e / BN_, k = e % BN_;
+      v[q] = *reinterpret_cast<const float4*>(Hblk + (long long)i * ld + k);
+    }
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+      const int e = (q * BASE_THREADS + threadIdx.x) * 4, i = e / BN_, k = e % BN_;
+      *reinterpret_cast<float4*>(sm + i * BLD + k) = v[q];
+      *reinterpret_cast<float4*>(sm + U_OFF + i * BLD + k) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  } else {
+    for (int e = threadIdx.x; e < BN_ * BN_; e += BASE_THREADS) {
+      const int i = e / BN_, k = e % BN_;
+      float v = 0.f;
+      if (i < n && k < n) v = (i <= k) ? Hblk[(long long)i * ld + k] : 0.f;
+      else if (i == k) v = 1.f;  // identity padding at the end
+      sm[i * BLD + k] = v;
+      sm[U_OFF + i * BLD + k] = 0.f;
+    }
   }
   __syncthreads();
   if (bad) return;
-  if (!base_rec<BN_>(A, U, V, 0, status, index0, &fail)) return;
-  for (int e = threadIdx.x; e < n * n; e += BASE_THREADS) {
-    const int i = e / n, k = e % n;
-    Ublk[(long long)i * ld + k] = (i <= k) ? U[i * BLD + k] : 0.f;
+  if (!base_rec<BN_>(0, status, index0, &fail)) return;
+  if (vec) {
+    constexpr int kPer = BN_ * BN_ / 4 / BASE_THREADS;
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+      const int e = (q * BASE_THREADS + threadIdx.x) * 4, i = e / BN_, k = e % BN_;
+      float4 v = *reinterpret_cast<const float4*>(sm + U_OFF + i * BLD + k);
+      // The shared U is zero below the diagonal already; the mask makes the output's lower
+      // triangle independent of that.
+      if (k + 0 < i) v.x = 0.f;
+      if (k + 1 < i) v.y = 0.f;
+      if (k + 2 < i) v.z = 0.f;
+      if (k + 3 < i) v.w = 0.f;
+      *reinterpret_cast<float4*>(Ublk + (long long)i * ld + k) = v;
+    }
+  } else {
+    for (int e = threadIdx.x; e < n * n; e += BASE_THREADS) {
+      const int i = e / n, k = e % n;
+      Ublk[(long long)i * ld + k] = (i <= k) ? sm[U_OFF + i * BLD + k] : 0.f;
+    }
   }
 }
 
@@ -346,7 +399,7 @@ int prep_zero_lower(float* U, int d, cudaStream_t stream) {
 
 int prep_base_block(float* Hblk, float* Ublk, int n, int ld, int index0, int32_t* status,
                     cudaStream_t stream) {
-  const size_t smem = (2 * (size_t)kPrepBase * BLD + 32 * VLD) * sizeof(float);
+  const size_t smem = 2 * (size_t)kPrepBase * BLD * sizeof(float);
   if (ensure_smem_attr(reinterpret_cast<const void*>(base_block_kernel), (int)smem) != 0)
     return GPTQ_ERR_CUDA;
   base_block_kernel<<<1, BASE_THREADS, smem, stream>>>(Hblk, Ublk, n, ld, index0, status);
