@@ -16,8 +16,9 @@
 // lane s of a row holds the four contiguous columns 4s..4s+3, so one row of U is read with
 // float4 loads, the remaining columns are spread evenly over the lanes, and chunks that are
 // already quantized are skipped uniformly. For column j the owner lane's value is broadcast
-// inside its 8-lane group, the group evaluates the quantizer, and the owner stores the code and
-// the error. The block's U (128 x 128, zero below the diagonal as gptq_prepare_hinv writes it)
+// inside its 8-lane group, the group evaluates the quantizer, and the owner keeps the code and
+// the error in registers; when a chunk is done every lane stores its four codes (one 32-bit
+// word) and errors (one float4). The block's U (128 x 128, zero below the diagonal as gptq_prepare_hinv writes it)
 // arrives in shared memory with one TMA copy; 1/U_jj is computed from it.
 #include <float.h>
 
@@ -33,9 +34,18 @@ constexpr int ROWS_PER_WARP = 4;
 constexpr int LANES_PER_ROW = 8;
 constexpr int SW_SMEM = BLK * BLK * 4 + BLK * 4 + 64;
 
-__device__ __forceinline__ float quant_code(float w, float s, float z, float maxq) {
-  const float q = rintf(__fdiv_rn(w, s)) + z;
-  return fminf(fmaxf(q, 0.0f), maxq);
+// q = clamp(rne(w / s) + z, 0, maxq) with the quotient rounded as in IEEE fp32 division, but
+// formed as a multiplication by rs = 1/s (correctly rounded) wherever that cannot change the
+// rounding. t = w * rs is within
+// 3 * 2^-24 |w/s| (two roundings and the reciprocal's) of the correctly rounded quotient, so
+// rint(t) equals rint(w / s) unless t lies within that distance of a rounding boundary
+// (k + 1/2); only then is the quotient formed exactly. The margin used, 2^-21 |t|, covers the
+// bound with room to spare.
+__device__ __forceinline__ float quant_code_rcp(float w, float s, float rs, float z, float maxq) {
+  float t = w * rs;
+  float r = rintf(t);
+  if (fabsf(fabsf(t - r) - 0.5f) <= 4.76837158e-7f * fabsf(t)) r = rintf(__fdiv_rn(w, s));
+  return fminf(fmaxf(r + z, 0.0f), maxq);
 }
 
 __device__ __forceinline__ void asym_params(float mn, float mx, float maxq, float& s, float& z) {
@@ -107,6 +117,11 @@ sweep_block_kernel(const __grid_constant__ CUtensorMap tmap_u, const float* __re
     s = scales[rsafe];
     z = zeros[rsafe];
   }
+  float rs = __frcp_rn(s);
+  // Group sizes divide 128 and are multiples of 4, hence powers of two: a group starts where
+  // the column's low bits are zero.
+  const bool grouped = g > 0;
+  const int gmask = grouped ? g - 1 : 0;
   const bool landed = gptq::mbar_wait(bar, 0, &abort_flag);
   if (!__syncthreads_and(landed)) {  // the copy did not arrive in time: report, touch nothing
     if (tid == 0) gptq::set_status(status, GPTQ_ERR_TIMEOUT, 3);
@@ -117,15 +132,17 @@ sweep_block_kernel(const __grid_constant__ CUtensorMap tmap_u, const float* __re
 
   float* erow = Err + (long long)rsafe * d + col0;
   uint8_t* crow = codes + (long long)rsafe * d + col0;
+  const bool codes_vec = (reinterpret_cast<uintptr_t>(codes) & 3) == 0 && (d & 3) == 0;
   bool finite = true;
 #pragma unroll
   for (int c = 0; c < 4; ++c) {                  // 32-column chunks
+    float qk[4], ek[4];                          // this lane's four codes and errors of chunk c
 #pragma unroll 1
     for (int so = 0; so < 8; ++so) {             // owner sub-lane within the chunk
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int j = 32 * c + 4 * so + e;
-        if (g > 0 && (j % g) == 0) {
+        if (grouped && (j & gmask) == 0) {
           float a = sym ? 0.f : FLT_MAX, b = -FLT_MAX;
 #pragma unroll
           for (int c2 = 0; c2 < 4; ++c2)
@@ -146,6 +163,7 @@ sweep_block_kernel(const __grid_constant__ CUtensorMap tmap_u, const float* __re
             b = group8_max(b);
             asym_params(a, b, maxq, s, z);
           }
+          rs = __frcp_rn(s);
           if (sub == 0 && live) {
             const long long gi = (long long)row * G + (col0 + j) / g;
             scales[gi] = s;
@@ -153,11 +171,11 @@ sweep_block_kernel(const __grid_constant__ CUtensorMap tmap_u, const float* __re
           }
         }
         const float wj = __shfl_sync(0xffffffffu, w[4 * c + e], grp | so);
-        const float qv = quant_code(wj, s, z, maxq);
+        const float qv = quant_code_rcp(wj, s, rs, z, maxq);
         const float err = (wj - s * (qv - z)) * invd[j];
-        if (sub == so && live) {
-          crow[j] = (uint8_t)qv;
-          erow[j] = err;
+        if (sub == so) {
+          qk[e] = qv;
+          ek[e] = err;
         }
         finite = finite && (fabsf(err) <= FLT_MAX);
         // w_k -= err * U_jk for the columns of chunks c..3 (U_jk = 0 for k < j).
@@ -170,6 +188,19 @@ sweep_block_kernel(const __grid_constant__ CUtensorMap tmap_u, const float* __re
           w[4 * c2 + 2] = fmaf(-err, u.z, w[4 * c2 + 2]);
           w[4 * c2 + 3] = fmaf(-err, u.w, w[4 * c2 + 3]);
         }
+      }
+    }
+    // Chunk done: each lane stores its four columns 32c + 4 sub .. +3 at once.
+    if (live) {
+      const int k0 = 32 * c + 4 * sub;
+      *reinterpret_cast<float4*>(erow + k0) = make_float4(ek[0], ek[1], ek[2], ek[3]);
+      const uint32_t packed = (uint32_t)qk[0] | ((uint32_t)qk[1] << 8) |
+                              ((uint32_t)qk[2] << 16) | ((uint32_t)qk[3] << 24);
+      if (codes_vec) {
+        *reinterpret_cast<uint32_t*>(crow + k0) = packed;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) crow[k0 + e] = (uint8_t)(packed >> (8 * e));
       }
     }
   }
