@@ -71,8 +71,44 @@ int split_point(int n) {  // a multiple of 128 near n/2, with 0 < m < n
   return m;
 }
 
+// Side streams for work off the recursion's critical path. V = T U22 of a split needs only T,
+// so it runs on a side stream while the caller's stream goes on with S and the recursion on S,
+// and the caller's stream waits for it before U12 = -U11 V. One stream and one fork/join event
+// pair per recursion depth, per device and per host thread, created on first use and kept for
+// the thread's lifetime. A thread issues its calls in order, so a pair is never in use by two
+// splits at once; event record/wait pairs are captured into CUDA graphs as dependencies.
+constexpr int kSideDepth = 24;
+constexpr int kSideDevices = 64;
+
+struct SideStreams {
+  bool ready = false;
+  cudaStream_t stream[kSideDepth] = {};
+  cudaEvent_t fork[kSideDepth] = {};
+  cudaEvent_t join[kSideDepth] = {};
+};
+
+SideStreams* side_streams() {
+  thread_local SideStreams per_device[kSideDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kSideDevices) return nullptr;
+  SideStreams& ss = per_device[dev];
+  if (!ss.ready) {
+    for (int i = 0; i < kSideDepth; ++i) {
+      if (cudaStreamCreateWithFlags(&ss.stream[i], cudaStreamNonBlocking) != cudaSuccess ||
+          cudaEventCreateWithFlags(&ss.fork[i], cudaEventDisableTiming) != cudaSuccess ||
+          cudaEventCreateWithFlags(&ss.join[i], cudaEventDisableTiming) != cudaSuccess)
+        return nullptr;
+    }
+    ss.ready = true;
+  }
+  return &ss;
+}
+
 // U block [off, off+n) from the damped, permuted Hessian block of the same rows/columns.
-int rec_prepare(float* H, float* U, int d, int off, int n, int32_t* st, cudaStream_t s) {
+// The factors U22 and U11 are upper triangular with exact zeros below the diagonal, so the
+// products with them skip the k-ranges where their terms vanish.
+int rec_prepare(float* H, float* U, int d, int off, int n, int depth, SideStreams* side,
+                int32_t* st, cudaStream_t s) {
   using namespace gptq_host;
   const long long ld = d;
   if (n <= kPrepBase) return prep_base_block(H + off * ld + off, U + off * ld + off, n, d, off, st, s);
@@ -84,19 +120,32 @@ int rec_prepare(float* H, float* U, int d, int off, int n, int32_t* st, cudaStre
   float* U12 = U + (long long)off * ld + off + m;
   float* U22 = U + (long long)(off + m) * ld + off + m;
   int rc;
-  if ((rc = rec_prepare(H, U, d, off + m, n2, st, s))) return rc;
-  // T = B U22^T -> U12 slot
-  if ((rc = gemm_f32(m, n2, n2, 1.f, Bblk, ld, false, U22, ld, true, 0.f, U12, ld, false, st, s)))
+  if ((rc = rec_prepare(H, U, d, off + m, n2, depth + 1, side, st, s))) return rc;
+  // T = B U22^T -> U12 slot (U22^T is lower triangular)
+  if ((rc = gemm_f32(m, n2, n2, 1.f, Bblk, ld, false, U22, ld, true, 0.f, U12, ld, false, st, s,
+                     kTriBLower)))
     return rc;
+  // V = T U22 -> B slot (B is no longer needed), on the side stream when there is one
+  const bool fork = side != nullptr && depth < kSideDepth;
+  cudaStream_t vs = s;
+  if (fork) {
+    vs = side->stream[depth];
+    if (cudaEventRecord(side->fork[depth], s) != cudaSuccess ||
+        cudaStreamWaitEvent(vs, side->fork[depth], 0) != cudaSuccess)
+      return GPTQ_ERR_CUDA;
+  }
+  if ((rc = gemm_f32(m, n2, n2, 1.f, U12, ld, false, U22, ld, false, 0.f, Bblk, ld, false, st, vs,
+                     kTriBUpper)))
+    return rc;
+  if (fork && cudaEventRecord(side->join[depth], vs) != cudaSuccess) return GPTQ_ERR_CUDA;
   // S = A - T T^T (upper triangle) in place of A
   if ((rc = gemm_f32(m, m, n2, -1.f, U12, ld, false, U12, ld, true, 1.f, Ablk, ld, true, st, s)))
     return rc;
-  if ((rc = rec_prepare(H, U, d, off, m, st, s))) return rc;
-  // V = T U22 -> B slot (B is no longer needed)
-  if ((rc = gemm_f32(m, n2, n2, 1.f, U12, ld, false, U22, ld, false, 0.f, Bblk, ld, false, st, s)))
-    return rc;
-  // U12 = -U11 V
-  return gemm_f32(m, n2, m, -1.f, U11, ld, false, Bblk, ld, false, 0.f, U12, ld, false, st, s);
+  if ((rc = rec_prepare(H, U, d, off, m, depth + 1, side, st, s))) return rc;
+  if (fork && cudaStreamWaitEvent(s, side->join[depth], 0) != cudaSuccess) return GPTQ_ERR_CUDA;
+  // U12 = -U11 V (U11 is upper triangular)
+  return gemm_f32(m, n2, m, -1.f, U11, ld, false, Bblk, ld, false, 0.f, U12, ld, false, st, s,
+                  kTriAUpper);
 }
 
 struct SweepCtx {
@@ -204,7 +253,7 @@ int gptq_prepare_hinv(float* H, int64_t d_in, const gptq_params* p, float* U, in
   }
   if (!rc) rc = prep_dead_damp(H, dead, d, p->percdamp, dev_status, s);
   if (!rc) rc = prep_zero_lower(U, d, s);
-  if (!rc) rc = rec_prepare(H, U, d, 0, d, dev_status, s);
+  if (!rc) rc = rec_prepare(H, U, d, 0, d, 0, side_streams(), dev_status, s);
   return rc ? GPTQ_ERR_CUDA : GPTQ_OK;
 }
 

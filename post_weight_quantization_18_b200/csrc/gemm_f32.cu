@@ -16,7 +16,7 @@ __global__ void __launch_bounds__(THREADS)
 gemm_f32_simt_kernel(int M, int N, int K, float alpha, const float* __restrict__ A, long long lda,
                      int transA, const float* __restrict__ B, long long ldb, int transB,
                      float beta, float* __restrict__ C, long long ldc, int upper_only,
-                     const int32_t* status) {
+                     int tri, const int32_t* status) {
   __shared__ __align__(16) float As[2][TK][TM + 4];
   __shared__ __align__(16) float Bs[2][TK][TN + 4];
   if (gptq::status_bad(status)) return;
@@ -57,11 +57,13 @@ gemm_f32_simt_kernel(int M, int N, int K, float alpha, const float* __restrict__
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
 
-  const int nk = (K + TK - 1) / TK;
-  if (nk > 0) load(0, 0);
+  int k_lo, k_hi;
+  gptq_host::tri_k_range(tri, m0, n0, n0 + TN, K, k_lo, k_hi);
+  const int kt0 = k_lo / TK, nk = (k_hi + TK - 1) / TK;
+  if (kt0 < nk) load(0, kt0 * TK);
   __syncthreads();
-  for (int kt = 0; kt < nk; ++kt) {
-    const int cur = kt & 1;
+  for (int kt = kt0; kt < nk; ++kt) {
+    const int cur = (kt - kt0) & 1;
     if (kt + 1 < nk) load(cur ^ 1, (kt + 1) * TK);
 #pragma unroll
     for (int kk = 0; kk < TK; ++kk) {
@@ -106,7 +108,7 @@ __global__ void __launch_bounds__(256)
 gemm_f32_small_kernel(int M, int N, int K, float alpha, const float* __restrict__ A, long long lda,
                       int transA, const float* __restrict__ B, long long ldb, int transB,
                       float beta, float* __restrict__ C, long long ldc, int upper_only,
-                      const int32_t* status) {
+                      int tri, const int32_t* status) {
   __shared__ float As[SK][ST + 1];  // As[k][m]
   __shared__ float Bs[SK][ST + 1];  // Bs[k][n]
   if (gptq::status_bad(status)) return;
@@ -114,7 +116,9 @@ gemm_f32_small_kernel(int M, int N, int K, float alpha, const float* __restrict_
   if (upper_only && m0 > n0 + ST - 1) return;
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   float acc[2][2] = {};
-  for (int k0 = 0; k0 < K; k0 += SK) {
+  int k_lo, k_hi;
+  gptq_host::tri_k_range(tri, m0, n0, n0 + ST, K, k_lo, k_hi);
+  for (int k0 = k_lo / SK * SK; k0 < k_hi; k0 += SK) {
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
       const int e = tid + 256 * r;  // 1024 elements per operand slab
@@ -160,11 +164,12 @@ namespace gptq_host {
 
 int gemm_f32_small(int M, int N, int K, float alpha, const float* A, long long lda, bool transA,
                    const float* B, long long ldb, bool transB, float beta, float* C,
-                   long long ldc, bool upper_only, const int32_t* status, cudaStream_t stream) {
+                   long long ldc, bool upper_only, const int32_t* status, cudaStream_t stream,
+                   int tri) {
   dim3 grid((N + ST - 1) / ST, (M + ST - 1) / ST);
   gemm_f32_small_kernel<<<grid, 256, 0, stream>>>(M, N, K, alpha, A, lda, transA ? 1 : 0, B, ldb,
                                                   transB ? 1 : 0, beta, C, ldc,
-                                                  upper_only ? 1 : 0, status);
+                                                  upper_only ? 1 : 0, tri, status);
   return cudaGetLastError() == cudaSuccess ? 0 : GPTQ_ERR_CUDA;
 }
 
@@ -172,12 +177,12 @@ int gemm_f32_small(int M, int N, int K, float alpha, const float* A, long long l
 // 16-byte aligned) and for K = 0; everything else goes to the tcgen05 3xTF32 kernel.
 int gemm_f32_simt(int M, int N, int K, float alpha, const float* A, long long lda, bool transA,
                   const float* B, long long ldb, bool transB, float beta, float* C, long long ldc,
-                  bool upper_only, const int32_t* status, cudaStream_t stream) {
+                  bool upper_only, const int32_t* status, cudaStream_t stream, int tri) {
   if (M <= 0 || N <= 0) return 0;
   dim3 grid((N + TN - 1) / TN, (M + TM - 1) / TM);
   gemm_f32_simt_kernel<<<grid, THREADS, 0, stream>>>(M, N, K, alpha, A, lda, transA ? 1 : 0, B,
                                                      ldb, transB ? 1 : 0, beta, C, ldc,
-                                                     upper_only ? 1 : 0, status);
+                                                     upper_only ? 1 : 0, tri, status);
   return cudaGetLastError() == cudaSuccess ? 0 : GPTQ_ERR_CUDA;
 }
 
@@ -187,19 +192,19 @@ namespace gptq_host {
 
 int gemm_f32(int M, int N, int K, float alpha, const float* A, long long lda, bool transA,
              const float* B, long long ldb, bool transB, float beta, float* C, long long ldc,
-             bool upper_only, const int32_t* status, cudaStream_t stream) {
+             bool upper_only, const int32_t* status, cudaStream_t stream, int tri) {
   if (M <= 0 || N <= 0) return 0;
   // Outputs of at most four 128 x 128 tiles (the bottom levels of the U recursion) finish
   // sooner on many small CUDA-core tiles than through the tensor-core pipeline's fill latency
   // (measured: 128^3 8 us vs 12 us, 256^3 14 us vs 16 us); larger ones go to tcgen05 (3xTF32).
   if ((long long)M * N <= 4LL * 128 * 128)
     return gemm_f32_small(M, N, K, alpha, A, lda, transA, B, ldb, transB, beta, C, ldc,
-                          upper_only, status, stream);
+                          upper_only, status, stream, tri);
   if (gemm_tf32x3_supported(M, N, K, A, lda, B, ldb, C, ldc))
     return gemm_tf32x3(M, N, K, alpha, A, lda, transA, B, ldb, transB, beta, C, ldc, upper_only,
-                       status, stream);
+                       status, stream, tri);
   return gemm_f32_simt(M, N, K, alpha, A, lda, transA, B, ldb, transB, beta, C, ldc, upper_only,
-                       status, stream);
+                       status, stream, tri);
 }
 
 }  // namespace gptq_host

@@ -41,6 +41,7 @@ struct GemmArgs {
   long long ldc;
   int a_mn, b_mn;      // 1: operand is MN-major in memory
   int upper_only;
+  int tri;             // kTri* flags: triangular operands, per-tile k-ranges
   int tiles_m, tiles_n, n_tiles;
   const int32_t* status;
   int32_t* status_w;
@@ -64,6 +65,19 @@ __device__ __forceinline__ void tile_of(int t, const GemmArgs& a, int& tm, int& 
 
 __device__ __forceinline__ bool tile_live(int tm, int tn, const GemmArgs& a) {
   return !a.upper_only || (tm * BM <= tn * BN + BN - 1);
+}
+
+// K blocks [kb0, kb1) of a tile: the blocks that can hold nonzero terms under the operands'
+// triangular structure. Never empty (an extra block only adds exact zeros), so that every tile
+// produces at least one accumulator for the epilogue. Every warp role derives the same range.
+__device__ __forceinline__ void tile_kb(int tm, int tn, const GemmArgs& a, int nkb, int& kb0,
+                                        int& kb1) {
+  int k_lo, k_hi;
+  gptq_host::tri_k_range(a.tri, tm * BM, tn * BN, tn * BN + BN, a.K, k_lo, k_hi);
+  kb0 = k_lo / BK;
+  kb1 = (k_hi + BK - 1) / BK;
+  if (kb0 > nkb - 1) kb0 = nkb - 1;
+  if (kb1 <= kb0) kb1 = kb0 + 1;
 }
 
 __global__ void __launch_bounds__(THREADS, 1)
@@ -120,7 +134,9 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
           int tm, tn;
           tile_of(t, args, tm, tn);
           if (!tile_live(tm, tn, args)) continue;
-          for (int kb = 0; kb < nkb; ++kb) {  // chunks of one tile are consecutive k-blocks
+          int kb0, kb1;
+          tile_kb(tm, tn, args, nkb, kb0, kb1);
+          for (int kb = kb0; kb < kb1; ++kb) {  // chunks of one tile are consecutive k-blocks
             if (!gptq::mbar_wait(&empty[stage], phase ^ 1, abort_flag)) break;
             uint8_t* sa = smem + stage * STAGE_BYTES;
             uint8_t* sb = sa + 2 * TILE_BYTES;
@@ -155,9 +171,11 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
           int tm, tn;
           tile_of(t, args, tm, tn);
           if (!tile_live(tm, tn, args)) continue;
+          int kb0, kb1;
+          tile_kb(tm, tn, args, nkb, kb0, kb1);
           bool ok = true;
-          for (int kc = 0; kc < nkb && ok; kc += KCB) {
-            const int kc1 = min(nkb, kc + KCB);
+          for (int kc = kb0; kc < kb1 && ok; kc += KCB) {
+            const int kc1 = min(kb1, kc + KCB);
             if (!gptq::mbar_wait(&acc_empty[buf], acc_phase ^ 1, abort_flag)) { ok = false; break; }
             gptq::tc_fence_after();
             const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
@@ -195,7 +213,9 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
         int tm, tn;
         tile_of(t, args, tm, tn);
         if (!tile_live(tm, tn, args)) continue;
-        for (int kb = 0; kb < nkb; ++kb) {
+        int kb0, kb1;
+        tile_kb(tm, tn, args, nkb, kb0, kb1);
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!gptq::mbar_wait(&full[stage], phase, abort_flag)) break;
           uint8_t* st = smem + stage * STAGE_BYTES;
 #pragma unroll
@@ -229,9 +249,11 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
         int tm, tn;
         tile_of(t, args, tm, tn);
         if (!tile_live(tm, tn, args)) continue;
+        int kb0, kb1;
+        tile_kb(tm, tn, args, nkb, kb0, kb1);
         bool ok = true;
-        for (int kc = 0; kc < nkb; kc += KCB) {
-        const float beta = (kc == 0) ? args.beta : 1.0f;  // later chunks fold into C
+        for (int kc = kb0; kc < kb1; kc += KCB) {
+        const float beta = (kc == kb0) ? args.beta : 1.0f;  // later chunks fold into C
         if (!gptq::mbar_wait(&acc_full[buf], acc_phase, abort_flag)) { ok = false; break; }
         gptq::tc_fence_after();
         const int row = tm * BM + quarter * 32 + lane;
@@ -309,7 +331,7 @@ bool gemm_tf32x3_supported(int M, int N, int K, const float* A, long long lda, c
 // op(B) is K x N: transB=false -> B[k*ldb + n] (MN-major); transB=true -> B[n*ldb + k] (K-major).
 int gemm_tf32x3(int M, int N, int K, float alpha, const float* A, long long lda, bool transA,
                 const float* B, long long ldb, bool transB, float beta, float* C, long long ldc,
-                bool upper_only, const int32_t* status, cudaStream_t stream) {
+                bool upper_only, const int32_t* status, cudaStream_t stream, int tri) {
   CUtensorMap ta, tb;
   const CUtensorMapDataType f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
   const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;               // K-major tiles
@@ -332,6 +354,7 @@ int gemm_tf32x3(int M, int N, int K, float alpha, const float* A, long long lda,
   a.a_mn = transA ? 1 : 0;
   a.b_mn = transB ? 0 : 1;
   a.upper_only = upper_only ? 1 : 0;
+  a.tri = tri;
   a.tiles_m = (M + BM - 1) / BM;
   a.tiles_n = (N + BN - 1) / BN;
   a.n_tiles = a.tiles_m * a.tiles_n;

@@ -13,21 +13,43 @@ int syrk_bf16_upper(float* H, int d, long long ldh, const void* X, long long n_t
 
 // ---- fp32 GEMM: C = alpha * op(A) op(B) + beta * C, row-major; op(A) is M x K, op(B) K x N.
 // upper_only: only elements with row <= col of C are written (the rest is left untouched).
+// tri: triangular structure of the operands (kTri* flags below); each output tile then runs
+// only over the k-range where its terms can be nonzero. Terms outside that range must be
+// exact zeros, so skipping them leaves the result unchanged.
+enum : int {
+  kTriNone = 0,
+  kTriAUpper = 1,  // op(A)[m][k] = 0 for k < m
+  kTriBUpper = 2,  // op(B)[k][n] = 0 for k > n
+  kTriBLower = 4,  // op(B)[k][n] = 0 for k < n
+};
+// [k_lo, k_hi) of an output tile with rows from m0 and columns [n0, n_end), for inner size K.
+__host__ __device__ inline void tri_k_range(int tri, int m0, int n0, int n_end, int K, int& k_lo,
+                                            int& k_hi) {
+  k_lo = 0;
+  k_hi = K;
+  if ((tri & kTriAUpper) && m0 > k_lo) k_lo = m0;
+  if ((tri & kTriBLower) && n0 > k_lo) k_lo = n0;
+  if ((tri & kTriBUpper) && n_end < k_hi) k_hi = n_end;
+}
+
 int gemm_f32(int M, int N, int K, float alpha, const float* A, long long lda, bool transA,
              const float* B, long long ldb, bool transB, float beta, float* C, long long ldc,
-             bool upper_only, const int32_t* status, cudaStream_t stream);
+             bool upper_only, const int32_t* status, cudaStream_t stream, int tri = kTriNone);
 
 int gemm_f32_simt(int M, int N, int K, float alpha, const float* A, long long lda, bool transA,
                   const float* B, long long ldb, bool transB, float beta, float* C, long long ldc,
-                  bool upper_only, const int32_t* status, cudaStream_t stream);
+                  bool upper_only, const int32_t* status, cudaStream_t stream,
+                  int tri = kTriNone);
 int gemm_f32_small(int M, int N, int K, float alpha, const float* A, long long lda, bool transA,
                    const float* B, long long ldb, bool transB, float beta, float* C,
-                   long long ldc, bool upper_only, const int32_t* status, cudaStream_t stream);
+                   long long ldc, bool upper_only, const int32_t* status, cudaStream_t stream,
+                   int tri = kTriNone);
 bool gemm_tf32x3_supported(int M, int N, int K, const float* A, long long lda, const float* B,
                            long long ldb, const float* C, long long ldc);
 int gemm_tf32x3(int M, int N, int K, float alpha, const float* A, long long lda, bool transA,
                 const float* B, long long ldb, bool transB, float beta, float* C, long long ldc,
-                bool upper_only, const int32_t* status, cudaStream_t stream);
+                bool upper_only, const int32_t* status, cudaStream_t stream,
+                int tri = kTriNone);
 
 // ---- prepare ----
 int prep_permute_sym(const float* H, float* Hp, const int32_t* perm, int d, cudaStream_t stream);
