@@ -125,8 +125,9 @@ __global__ void zero_lower_kernel(float* U, int d) {
 //   128 -> 64 -> 32 -> 16-column leaves. Each split does the four block products of the host
 //   recursion on the tensor cores (warp-level m16n8k8 TF32 with the three-term hi/lo split, so
 //   the products carry fp32 accuracy), skipping the k-ranges where the triangular operand is
-//   zero and computing only the upper tiles of the symmetric update. A leaf is factored and
-//   inverted by one warp in registers (no block barriers inside).
+//   zero and computing only the upper tiles of the symmetric update. A 32-column node (two
+//   leaves and its four 16 x 16 products) runs on one warp without block barriers; a leaf is
+//   factored and inverted in registers.
 // A block smaller than 128 is padded at its end with the identity: the padded factor is block
 // diagonal, so the leading n x n part is unchanged.
 constexpr int BASE_THREADS = 512;
@@ -209,29 +210,35 @@ GPTQ_DEV void mma_m16n8k8_tf32(float (&d)[4], const uint32_t (&a)[4], uint32_t b
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// C (m x m) = alpha * X Y' + beta * C on shared-memory blocks (offsets into the dynamic shared
-// array, pitch BLD), Y' = Y (ty = 0, Y[k][n]) or Y^T (ty = 1, Y[n][k]). Warps w0 .. w0+nw-1
-// take 16 x 16 output tiles in turn. Each product x*y is formed as
-// hi(x)hi(y) + hi(x)lo(y) + lo(x)hi(y) with hi the operand's top 19 bits (TF32) and lo the rest.
-__device__ __noinline__ void block_mma(int m, int c_off, int x_off, int y_off, int ty,
-                                       float alpha, float beta, int tri, int w0, int nw) {
+// C (M x M) = alpha * X Y' + beta * C on shared-memory blocks (offsets into the dynamic shared
+// array, pitch BLD), Y' = Y^T (Y read as Y[n][k]) for the transposed kinds and Y (Y[k][n])
+// otherwise. Warps w0 .. w0+nw-1 take 16 x 16 output tiles in turn. Each product x*y is formed
+// as hi(x)hi(y) + hi(x)lo(y) + lo(x)hi(y) with hi the operand's top 19 bits (TF32) and lo the
+// rest. One instance per (M, TRI), so that the k-loop is unrolled and the operand layout fixed
+// at compile time.
+template <int M, int TRI>
+__device__ __noinline__ void block_mma(int c_off, int x_off, int y_off, float alpha, float beta,
+                                       int w0, int nw) {
   extern __shared__ float sm[];
+  constexpr bool kYT = (TRI == kYUpperTransposed || TRI == kCUpperOnly);
+  constexpr int kTiles = M / 16;
   const int warp = (threadIdx.x >> 5) - w0, lane = threadIdx.x & 31;
   if (warp < 0 || warp >= nw) return;
   const int g = lane >> 2, t = lane & 3;
-  const int tiles = m >> 4;
   const float* X = sm + x_off;
   const float* Y = sm + y_off;
   float* C = sm + c_off;
-  for (int tile = warp; tile < tiles * tiles; tile += nw) {
-    const int i0 = (tile / tiles) * 16, n0 = (tile % tiles) * 16;
-    if (tri == kCUpperOnly && i0 > n0) continue;
-    int k_lo = 0, k_hi = m;
-    if (tri == kYUpperTransposed) k_lo = n0;
-    if (tri == kYUpper) k_hi = n0 + 16;
-    if (tri == kXUpper) k_lo = i0;
+  for (int tile = warp; tile < kTiles * kTiles; tile += nw) {
+    const int i0 = (tile / kTiles) * 16, n0 = (tile % kTiles) * 16;
+    if (TRI == kCUpperOnly && i0 > n0) continue;
+    int k_lo = 0, k_hi = M;
+    if (TRI == kYUpperTransposed) k_lo = n0;
+    if (TRI == kYUpper) k_hi = n0 + 16;
+    if (TRI == kXUpper) k_lo = i0;
     float hh[2][4] = {}, cross[2][4] = {};
-    for (int k0 = k_lo; k0 < k_hi; k0 += 8) {
+#pragma unroll
+    for (int k0 = 0; k0 < M; k0 += 8) {
+      if (k0 < k_lo || k0 >= k_hi) continue;
       const float xa[4] = {X[(i0 + g) * BLD + k0 + t], X[(i0 + g + 8) * BLD + k0 + t],
                            X[(i0 + g) * BLD + k0 + t + 4], X[(i0 + g + 8) * BLD + k0 + t + 4]};
       uint32_t ah[4], al[4];
@@ -243,8 +250,8 @@ __device__ __noinline__ void block_mma(int m, int c_off, int x_off, int y_off, i
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int n = n0 + 8 * h + g;
-        const float y0 = ty ? Y[n * BLD + k0 + t] : Y[(k0 + t) * BLD + n];
-        const float y1 = ty ? Y[n * BLD + k0 + t + 4] : Y[(k0 + t + 4) * BLD + n];
+        const float y0 = kYT ? Y[n * BLD + k0 + t] : Y[(k0 + t) * BLD + n];
+        const float y1 = kYT ? Y[n * BLD + k0 + t + 4] : Y[(k0 + t + 4) * BLD + n];
         const uint32_t bh0 = tf32_hi(y0), bh1 = tf32_hi(y1);
         mma_m16n8k8_tf32(cross[h], ah, tf32_lo(y0, bh0), tf32_lo(y1, bh1));
         mma_m16n8k8_tf32(cross[h], al, bh0, bh1);
@@ -262,13 +269,43 @@ __device__ __noinline__ void block_mma(int m, int c_off, int x_off, int y_off, i
   }
 }
 
+// Offsets of the blocks of one split: node [o, o+N) split at m = N/2.
+struct Split {
+  int Bb, Aa, U11, U12, U22;
+  __device__ Split(int o, int m)
+      : Bb(o * BLD + o + m),                 // A[o:o+m, o+m:o+N]
+        Aa(o * BLD + o),                     // A[o:o+m, o:o+m]
+        U11(U_OFF + o * BLD + o),
+        U12(U_OFF + o * BLD + o + m),
+        U22(U_OFF + (o + m) * BLD + o + m) {}
+};
+
+// A 32-column node [o, o+32) entirely on warp 0: two 16-column leaves and the four 16 x 16
+// products of the split, ordered by __syncwarp only. Returns -1 or the failing column (within
+// the node) of the first non-positive pivot; the value is the same on every lane of warp 0.
+__device__ __forceinline__ int node32_warp(int o) {
+  const Split sp(o, 16);
+  int bad = leaf16(o + 16);
+  if (bad >= 0) return 16 + bad;
+  block_mma<16, kYUpperTransposed>(sp.U12, sp.Bb, sp.U22, 1.f, 0.f, 0, 1);  // T = B U22^T
+  __syncwarp();
+  block_mma<16, kCUpperOnly>(sp.Aa, sp.U12, sp.U12, -1.f, 1.f, 0, 1);      // S = A - T T^T
+  block_mma<16, kYUpper>(sp.Bb, sp.U12, sp.U22, 1.f, 0.f, 0, 1);           // V = T U22
+  __syncwarp();
+  bad = leaf16(o);
+  if (bad >= 0) return bad;
+  block_mma<16, kXUpper>(sp.U12, sp.U11, sp.Bb, -1.f, 0.f, 0, 1);          // U12 = -U11 V
+  __syncwarp();
+  return -1;
+}
+
 template <int N>
 __device__ __forceinline__ bool base_rec(int o, int32_t* status, int index0, int* fail) {
-  if constexpr (N == kLeaf) {
+  if constexpr (N == 32) {
     if (threadIdx.x < 32) {
-      const int badj = leaf16(o);
-      if (badj >= 0 && threadIdx.x == 0) {
-        gptq::set_status(status, GPTQ_ERR_NOT_SPD, index0 + o + badj);
+      const int bad = node32_warp(o);
+      if (bad >= 0 && threadIdx.x == 0) {
+        gptq::set_status(status, GPTQ_ERR_NOT_SPD, index0 + o + bad);
         *fail = 1;
       }
     }
@@ -276,20 +313,16 @@ __device__ __forceinline__ bool base_rec(int o, int32_t* status, int index0, int
     return *fail == 0;
   } else {
     constexpr int m = N / 2;
-    const int Bb = o * BLD + o + m;             // A[o:o+m, o+m:o+N]
-    const int Aa = o * BLD + o;                 // A[o:o+m, o:o+m]
-    const int U11 = U_OFF + o * BLD + o;
-    const int U12 = U_OFF + o * BLD + o + m;
-    const int U22 = U_OFF + (o + m) * BLD + o + m;
+    const Split sp(o, m);
     if (!base_rec<m>(o + m, status, index0, fail)) return false;
-    block_mma(m, U12, Bb, U22, 1, 1.f, 0.f, kYUpperTransposed, 0, BASE_WARPS);  // T = B U22^T
+    block_mma<m, kYUpperTransposed>(sp.U12, sp.Bb, sp.U22, 1.f, 0.f, 0, BASE_WARPS);  // T
     __syncthreads();
     // S = A - T T^T (upper tiles) and V = T U22 both need only T: one barrier for the two.
-    block_mma(m, Aa, U12, U12, 1, -1.f, 1.f, kCUpperOnly, 0, BASE_WARPS / 2);
-    block_mma(m, Bb, U12, U22, 0, 1.f, 0.f, kYUpper, BASE_WARPS / 2, BASE_WARPS / 2);
+    block_mma<m, kCUpperOnly>(sp.Aa, sp.U12, sp.U12, -1.f, 1.f, 0, BASE_WARPS / 2);
+    block_mma<m, kYUpper>(sp.Bb, sp.U12, sp.U22, 1.f, 0.f, BASE_WARPS / 2, BASE_WARPS / 2);
     __syncthreads();
     if (!base_rec<m>(o, status, index0, fail)) return false;
-    block_mma(m, U12, U11, Bb, 0, -1.f, 0.f, kXUpper, 0, BASE_WARPS);          // U12 = -U11 V
+    block_mma<m, kXUpper>(sp.U12, sp.U11, sp.Bb, -1.f, 0.f, 0, BASE_WARPS);        // U12
     __syncthreads();
     return true;
   }
