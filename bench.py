@@ -52,6 +52,26 @@ def parse_args():
     return ap.parse_args()
 
 
+def syrk_traffic():
+    """DRAM bytes per launch of the SYRK kernel from its committed ncu summary, or None when the
+    kernel source has changed since the counters were taken (the summary records its hash)."""
+    import hashlib
+    import re
+    try:
+        with open(os.path.join(ROOT, "profiles", "syrk_bf16_llama7b_attn_proj.md")) as f:
+            text = f.read()
+        with open(os.path.join(ROOT, "post_weight_quantization_18_b200", "csrc",
+                               "syrk_bf16.cu"), "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()
+    except OSError:
+        return None
+    want = re.search(r"kernel_source_sha256:\s*([0-9a-f]{64})", text)
+    val = re.search(r"traffic_bytes_per_launch:\s*([0-9]+)", text)
+    if not want or not val or want.group(1) != digest:
+        return None
+    return int(val.group(1))
+
+
 def peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -465,7 +485,8 @@ def run_ours(args):
             "sweep_gbs": sweep_bytes / (quant_ms * 1e-3) / 1e9,
             "roofline": {"bound": "tensor", "kernel": "syrk_bf16_tcgen05_kernel",
                          "achieved": syrk_tflops, "peak": bf16, "unit": "TFLOP/s",
-                         "frac": syrk_tflops / bf16, "traffic": None,
+                         "frac": syrk_tflops / bf16,
+                         "traffic": syrk_traffic() if act.n_tokens == 262144 and d == 4096 else None,
                          "peak_source": f"{peak_kind} bf16 burst",
                          "algorithmic": f"d(d+1)N = {syrk_flops:.4g} flop per launch"},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,

@@ -158,6 +158,147 @@ gemm_f32_small_kernel(int M, int N, int K, float alpha, const float* __restrict_
   }
 }
 
+// Staged GEMMs for short inner dimensions: one CTA per 32 x 32 output tile, 256 threads. The
+// tile's k-range (after the triangular restriction) is brought into shared memory in chunks of
+// up to 256: every thread issues all of its 16-byte loads of a chunk before storing any, so a
+// chunk costs one memory round trip. Shared memory holds both operands k-major; an operand
+// stored with k contiguous in memory is transposed on the way in, with consecutive lanes on
+// consecutive rows so that the transposing stores hit distinct banks. Each of the 8 warps then takes an eighth of the chunk for
+// the whole tile (lane: 4 rows x 8 columns, operands read as float4) and the warps' partial
+// sums are added through shared memory at the end. Needs 16-byte aligned A and B, leading
+// dimensions and K multiples of 4.
+constexpr int GT = 32, GKC = 256, GPAD = 36, G_THREADS = 256;
+constexpr int G_SMEM = 2 * GKC * GPAD * 4;  // 72 KB: As[k][m] and Bs[k][n] of one chunk
+constexpr int G_PER = GT * GKC / 4 / G_THREADS;  // 16-byte granules per thread and operand (8)
+
+__global__ void __launch_bounds__(G_THREADS)
+gemm_f32_staged_kernel(int M, int N, int K, float alpha, const float* __restrict__ A,
+                       long long lda, int transA, const float* __restrict__ B, long long ldb,
+                       int transB, float beta, float* __restrict__ C, long long ldc,
+                       int upper_only, int tri, const int32_t* status) {
+  extern __shared__ __align__(16) float gsm[];
+  float* As = gsm;               // As[k][m], k relative to the chunk start
+  float* Bs = gsm + GKC * GPAD;  // Bs[k][n]
+  if (gptq::status_bad(status)) return;
+  const int m0 = blockIdx.y * GT, n0 = blockIdx.x * GT;
+  if (upper_only && m0 > n0 + GT - 1) return;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int r4 = 4 * (lane >> 2), c8 = 8 * (lane & 3);
+  int k_lo, k_hi;
+  gptq_host::tri_k_range(tri, m0, n0, n0 + GT, K, k_lo, k_hi);
+  k_lo &= ~3;
+  float acc[4][8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+
+  for (int kc = k_lo; kc < k_hi; kc += GKC) {
+    const int kn = min(GKC, k_hi - kc);  // a multiple of 4
+    const int kq = kn >> 2;
+    float4 va[G_PER], vb[G_PER];
+    // op(A)[m0 + mm][kc + kk] and op(B)[kc + kk][n0 + nn]; granules run along the contiguous
+    // direction of each operand in memory.
+#pragma unroll
+    for (int q = 0; q < G_PER; ++q) {
+      const int g = tid + q * G_THREADS;
+      va[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+      vb[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (g < GT * kq) {
+        if (!transA) {  // A[m][k]: granule = 4 consecutive k of row mm (lanes along m)
+          const int mm = g & 31, kk = 4 * (g >> 5);
+          if (m0 + mm < M)
+            va[q] = *reinterpret_cast<const float4*>(A + (long long)(m0 + mm) * lda + kc + kk);
+        } else {        // A[k][m]: granule = 4 consecutive m of row kk
+          const int kk = g >> 3, mm = 4 * (g & 7);
+          const float* src = A + (long long)(kc + kk) * lda + m0 + mm;
+          if (m0 + mm + 4 <= M) {
+            va[q] = *reinterpret_cast<const float4*>(src);
+          } else {
+            if (m0 + mm + 0 < M) va[q].x = src[0];
+            if (m0 + mm + 1 < M) va[q].y = src[1];
+            if (m0 + mm + 2 < M) va[q].z = src[2];
+          }
+        }
+        if (transB) {   // B[n][k]: granule = 4 consecutive k of row nn (lanes along n)
+          const int nn = g & 31, kk = 4 * (g >> 5);
+          if (n0 + nn < N)
+            vb[q] = *reinterpret_cast<const float4*>(B + (long long)(n0 + nn) * ldb + kc + kk);
+        } else {        // B[k][n]: granule = 4 consecutive n of row kk
+          const int kk = g >> 3, nn = 4 * (g & 7);
+          const float* src = B + (long long)(kc + kk) * ldb + n0 + nn;
+          if (n0 + nn + 4 <= N) {
+            vb[q] = *reinterpret_cast<const float4*>(src);
+          } else {
+            if (n0 + nn + 0 < N) vb[q].x = src[0];
+            if (n0 + nn + 1 < N) vb[q].y = src[1];
+            if (n0 + nn + 2 < N) vb[q].z = src[2];
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < G_PER; ++q) {
+      const int g = tid + q * G_THREADS;
+      if (g < GT * kq) {
+        if (!transA) {
+          const int mm = g & 31, kk = 4 * (g >> 5);
+          As[(kk + 0) * GPAD + mm] = va[q].x;
+          As[(kk + 1) * GPAD + mm] = va[q].y;
+          As[(kk + 2) * GPAD + mm] = va[q].z;
+          As[(kk + 3) * GPAD + mm] = va[q].w;
+        } else {
+          *reinterpret_cast<float4*>(As + (g >> 3) * GPAD + 4 * (g & 7)) = va[q];
+        }
+        if (transB) {
+          const int nn = g & 31, kk = 4 * (g >> 5);
+          Bs[(kk + 0) * GPAD + nn] = vb[q].x;
+          Bs[(kk + 1) * GPAD + nn] = vb[q].y;
+          Bs[(kk + 2) * GPAD + nn] = vb[q].z;
+          Bs[(kk + 3) * GPAD + nn] = vb[q].w;
+        } else {
+          *reinterpret_cast<float4*>(Bs + (g >> 3) * GPAD + 4 * (g & 7)) = vb[q];
+        }
+      }
+    }
+    __syncthreads();
+    const int kw = (kn + 7) >> 3;
+    const int kb = warp * kw, ke = min(kn, kb + kw);
+#pragma unroll 4
+    for (int k = kb; k < ke; ++k) {
+      const float4 a = *reinterpret_cast<const float4*>(As + k * GPAD + r4);
+      const float4 b0 = *reinterpret_cast<const float4*>(Bs + k * GPAD + c8);
+      const float4 b1 = *reinterpret_cast<const float4*>(Bs + k * GPAD + c8 + 4);
+      const float av[4] = {a.x, a.y, a.z, a.w};
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+    __syncthreads();  // the next chunk (or the reduction) overwrites the staging area
+  }
+  // Partial sums of the 8 warps -> shared memory (pitch 33), then 4 outputs per thread.
+  float* red = gsm;  // 8 x 32 x 33 floats, inside the staging area
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) red[(warp * GT + r4 + i) * 33 + c8 + j] = acc[i][j];
+  __syncthreads();
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int e = tid + q * G_THREADS, row = e >> 5, col = e & 31;
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) v += red[(w * GT + row) * 33 + col];
+    const int gm = m0 + row, gn = n0 + col;
+    if (gm >= M || gn >= N || (upper_only && gm > gn)) continue;
+    float* cp = C + (long long)gm * ldc + gn;
+    v *= alpha;
+    *cp = (beta == 0.f) ? v : fmaf(beta, *cp, v);
+  }
+}
+
 }  // namespace
 
 namespace gptq_host {
@@ -170,6 +311,26 @@ int gemm_f32_small(int M, int N, int K, float alpha, const float* A, long long l
   gemm_f32_small_kernel<<<grid, 256, 0, stream>>>(M, N, K, alpha, A, lda, transA ? 1 : 0, B, ldb,
                                                   transB ? 1 : 0, beta, C, ldc,
                                                   upper_only ? 1 : 0, tri, status);
+  return cudaGetLastError() == cudaSuccess ? 0 : GPTQ_ERR_CUDA;
+}
+
+bool gemm_f32_staged_supported(int K, const float* A, long long lda, const float* B,
+                               long long ldb) {
+  auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+  return K > 0 && (K % 4) == 0 && al16(A) && al16(B) && (lda % 4) == 0 && (ldb % 4) == 0;
+}
+
+int gemm_f32_staged(int M, int N, int K, float alpha, const float* A, long long lda, bool transA,
+                    const float* B, long long ldb, bool transB, float beta, float* C,
+                    long long ldc, bool upper_only, const int32_t* status, cudaStream_t stream,
+                    int tri) {
+  if (M <= 0 || N <= 0) return 0;
+  if (ensure_smem_attr(reinterpret_cast<const void*>(gemm_f32_staged_kernel), G_SMEM) != 0)
+    return GPTQ_ERR_CUDA;
+  dim3 grid((N + GT - 1) / GT, (M + GT - 1) / GT);
+  gemm_f32_staged_kernel<<<grid, G_THREADS, G_SMEM, stream>>>(
+      M, N, K, alpha, A, lda, transA ? 1 : 0, B, ldb, transB ? 1 : 0, beta, C, ldc,
+      upper_only ? 1 : 0, tri, status);
   return cudaGetLastError() == cudaSuccess ? 0 : GPTQ_ERR_CUDA;
 }
 
@@ -194,9 +355,13 @@ int gemm_f32(int M, int N, int K, float alpha, const float* A, long long lda, bo
              const float* B, long long ldb, bool transB, float beta, float* C, long long ldc,
              bool upper_only, const int32_t* status, cudaStream_t stream, int tri) {
   if (M <= 0 || N <= 0) return 0;
-  // Outputs of at most four 128 x 128 tiles (the bottom levels of the U recursion) finish
-  // sooner on many small CUDA-core tiles than through the tensor-core pipeline's fill latency
-  // (measured: 128^3 8 us vs 12 us, 256^3 14 us vs 16 us); larger ones go to tcgen05 (3xTF32).
+  // Products up to 512 x 512 x 512 (the lower levels of the U recursion) finish sooner on
+  // 32 x 32 CUDA-core tiles with the k-range staged in one round than through the tensor-core
+  // pipeline's fill latency (graph replay: 128^3 4.7 us vs 12.3 us, 256^3 6.4 vs 15.8, 512^3
+  // 16.3 vs 22.4); larger ones go to tcgen05 (3xTF32).
+  if (K <= 512 && (long long)M * N <= 512LL * 512 && gemm_f32_staged_supported(K, A, lda, B, ldb))
+    return gemm_f32_staged(M, N, K, alpha, A, lda, transA, B, ldb, transB, beta, C, ldc,
+                           upper_only, status, stream, tri);
   if ((long long)M * N <= 4LL * 128 * 128)
     return gemm_f32_small(M, N, K, alpha, A, lda, transA, B, ldb, transB, beta, C, ldc,
                           upper_only, status, stream, tri);

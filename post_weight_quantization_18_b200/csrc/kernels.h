@@ -44,6 +44,12 @@ int gemm_f32_small(int M, int N, int K, float alpha, const float* A, long long l
                    const float* B, long long ldb, bool transB, float beta, float* C,
                    long long ldc, bool upper_only, const int32_t* status, cudaStream_t stream,
                    int tri = kTriNone);
+bool gemm_f32_staged_supported(int K, const float* A, long long lda, const float* B,
+                               long long ldb);
+int gemm_f32_staged(int M, int N, int K, float alpha, const float* A, long long lda, bool transA,
+                    const float* B, long long ldb, bool transB, float beta, float* C,
+                    long long ldc, bool upper_only, const int32_t* status, cudaStream_t stream,
+                    int tri = kTriNone);
 bool gemm_tf32x3_supported(int M, int N, int K, const float* A, long long lda, const float* B,
                            long long ldb, const float* C, long long ldc);
 int gemm_tf32x3(int M, int N, int K, float alpha, const float* A, long long lda, bool transA,
