@@ -157,9 +157,13 @@ __device__ __noinline__ int leaf16(int o) {
 #pragma unroll
   for (int c = 0; c < N; ++c) a[c] = (lane < N && c >= lane) ? sm[(o + lane) * BLD + o + c] : 0.f;
   int badj = -1;
+  // dn: on lane j, the pivot of step j. The owner of the next pivot updates it from its own v,
+  // so the next step waits for one FMA rather than for this step's shuffles (same value as the
+  // shuffled update of a[j - 1] below).
+  float dn = a[N - 1];
 #pragma unroll
   for (int j = N - 1; j >= 0; --j) {
-    const float piv = __shfl_sync(0xffffffffu, a[j], j);
+    const float piv = __shfl_sync(0xffffffffu, dn, j);
     if (badj < 0 && !(piv > 0.f && piv <= 3.402823466e38f)) badj = j;
     // Reciprocal square root from the special-function unit (about 1 ulp, the order of the
     // factor's own fp32 rounding).
@@ -167,6 +171,7 @@ __device__ __noinline__ int leaf16(int o) {
     rinv[j] = inv;
     const float v = (lane < j) ? a[j] * inv : (lane == j ? piv * inv : 0.f);
     vrow[j] = v;
+    if (j > 0) dn = fmaf(-v, v, a[j - 1]);
 #pragma unroll
     for (int k = 0; k < j; ++k) {
       const float vk = __shfl_sync(0xffffffffu, v, k);

@@ -6,17 +6,21 @@
 // GEMM operands are X itself read "MN-major": element (t, i) sits at t*ldx + i.
 //
 // Design (one CTA per SM, persistent):
-//   * Work unit = (128 x 256 output tile with i-block <= j-block, token chunk). Only tiles that
-//     touch the upper triangle are scheduled; token chunks (split-K) are used only when the
-//     tiles alone cannot fill the SMs. Units are chunk-major so concurrently running CTAs
-//     share one L2-resident chunk of X.
-//   * warp 0: TMA producer — per 64-token k-block, two 64x64 boxes of X for the A tile (rows
-//     i0..i0+127) and four for the B tile (j0..j0+255), 128-byte swizzled, 4-stage ring.
-//   * warp 1: TMEM owner and MMA issuer — tcgen05.mma kind::f16, M=128, N=256, K=16, both
-//     operands MN-major; fp32 accumulators double-buffered in TMEM (2 x 256 columns).
+//   * Work unit = (256 x 256 output tile with i-block <= j-block, token chunk). Only tiles on or
+//     above the diagonal are scheduled; the token range is split into chunks of at most 8192
+//     tokens (and further only when the tiles alone cannot fill the SMs). Units are chunk-major
+//     so concurrently running CTAs share one L2-resident chunk of X.
+//   * warp 0: TMA producer — per 64-token k-block, four 64x64 boxes of X for the A tile (rows
+//     i0..i0+255) and four for the B tile (j0..j0+255), 128-byte swizzled, 3-stage ring.
+//   * warp 1: TMEM owner and MMA issuer — per 16-token step two tcgen05.mma kind::f16 of
+//     M=128, N=256, one per half of the A tile, sharing the B operand; both operands MN-major.
+//     The 256 x 256 fp32 accumulator fills TMEM (the halves at columns 0 and 256). A 256-row
+//     tile needs two thirds of the operand bytes per MMA of a 128-row one, which keeps the
+//     L2 -> SM feed and the TMA latency well inside what the ring covers.
 //   * warps 2-5: epilogue — tcgen05.ld 32 rows x 32 columns, scale by alpha, zero the strictly
 //     lower triangle, stage in 128B-swizzled smem and add into H with a TMA reduce-add
-//     (cp.reduce.async.bulk.tensor .add), which also clips the ragged edge of H.
+//     (cp.reduce.async.bulk.tensor .add), which also clips the ragged edge of H. The MMA warp
+//     starts the next unit once both halves are drained.
 //   * Every mbarrier wait is bounded; on timeout the CTA records GPTQ_ERR_TIMEOUT, leaves its
 //     loops, frees TMEM and returns.
 #include "common.cuh"
@@ -24,20 +28,21 @@
 
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int BM = 256, BN = 256, BK = 64, STAGES = 3;
+constexpr int MMA_M = 128;                        // rows per tcgen05.mma (two per k-step)
 constexpr int BOX = 64;                           // 64 bf16 = 128 B inner, 64 tokens outer
 constexpr int BOX_BYTES = BOX * BOX * 2;          // 8 KB
-constexpr int A_BYTES = 2 * BOX_BYTES;            // 16 KB
+constexpr int A_BYTES = 4 * BOX_BYTES;            // 32 KB
 constexpr int B_BYTES = 4 * BOX_BYTES;            // 32 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;    // 48 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;    // 64 KB
 constexpr int EPI_WARPS = 4;
 constexpr int EPI_TILE_BYTES = 32 * 32 * 4;       // 32 rows x 32 fp32 = 4 KB
 constexpr int EPI_BUFS = 2;
 constexpr int SMEM_DATA = STAGES * STAGE_BYTES + EPI_WARPS * EPI_BUFS * EPI_TILE_BYTES;
 constexpr int SMEM_BYTES = SMEM_DATA + 1024 /*align*/ + 256 /*barriers*/;
 constexpr int THREADS = 192;
-constexpr uint32_t TMEM_COLS = 512;               // two 128 x 256 fp32 accumulators
-constexpr uint32_t IDESC = gptq::instr_desc(/*bf16*/ 1, /*A MN*/ 1, /*B MN*/ 1, BM, BN);
+constexpr uint32_t TMEM_COLS = 512;               // the two 128 x 256 halves of the tile
+constexpr uint32_t IDESC = gptq::instr_desc(/*bf16*/ 1, /*A MN*/ 1, /*B MN*/ 1, MMA_M, BN);
 
 struct SyrkArgs {
   int d, n_ib, n_jb, n_tiles, n_split, kb_per_split, nkb_total;
@@ -47,10 +52,10 @@ struct SyrkArgs {
 };
 
 // Tile t (0..n_tiles-1) -> (ib, jb): column blocks jb in order, each with the row blocks
-// ib = 0..min(2*jb+1, n_ib-1) that reach the upper triangle.
+// ib = 0..jb on or above the diagonal.
 __device__ __forceinline__ void tile_coords(int t, int n_ib, int n_jb, int& ib, int& jb) {
   for (jb = 0; jb < n_jb; ++jb) {
-    int cnt = min(2 * jb + 2, n_ib);
+    int cnt = min(jb + 1, n_ib);
     if (t < cnt) { ib = t; return; }
     t -= cnt;
   }
@@ -68,8 +73,8 @@ syrk_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_x,
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SMEM_DATA);
   uint64_t* full = bars;                 // [STAGES]
   uint64_t* empty = bars + STAGES;       // [STAGES]
-  uint64_t* acc_full = bars + 2 * STAGES;    // [2]
-  uint64_t* acc_empty = bars + 2 * STAGES + 2;  // [2]
+  uint64_t* acc_full = bars + 2 * STAGES;       // accumulator complete
+  uint64_t* acc_empty = bars + 2 * STAGES + 1;  // accumulator drained
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* skip_flag = abort_flag + 1;
@@ -83,10 +88,8 @@ syrk_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_x,
       gptq::mbar_init(&full[s], 1);
       gptq::mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      gptq::mbar_init(&acc_full[b], 1);
-      gptq::mbar_init(&acc_empty[b], EPI_WARPS);
-    }
+    gptq::mbar_init(acc_full, 1);
+    gptq::mbar_init(acc_empty, EPI_WARPS);
     gptq::fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
@@ -121,8 +124,9 @@ syrk_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_x,
             uint8_t* sb = sa + A_BYTES;
             gptq::mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
             const int t = kb * BK;
-            gptq::tma_load_2d(sa, &tmap_x, &full[stage], ib * BM, t);
-            gptq::tma_load_2d(sa + BOX_BYTES, &tmap_x, &full[stage], ib * BM + BOX, t);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              gptq::tma_load_2d(sa + q * BOX_BYTES, &tmap_x, &full[stage], ib * BM + q * BOX, t);
 #pragma unroll
             for (int q = 0; q < 4; ++q)
               gptq::tma_load_2d(sb + q * BOX_BYTES, &tmap_x, &full[stage], jb * BN + q * BOX, t);
@@ -135,15 +139,14 @@ syrk_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_x,
       if (lane == 0) {
         int stage = 0;
         uint32_t phase = 0;
-        int buf = 0;
         uint32_t acc_phase = 0;
         for (long long u = blockIdx.x; u < args.n_units && !*abort_flag; u += gridDim.x) {
           const int split = (int)(u / args.n_tiles);
           const int kb0 = split * args.kb_per_split;
           const int kb1 = min(args.nkb_total, kb0 + args.kb_per_split);
-          if (!gptq::mbar_wait(&acc_empty[buf], acc_phase ^ 1, abort_flag)) break;
+          if (!gptq::mbar_wait(acc_empty, acc_phase ^ 1, abort_flag)) break;
           gptq::tc_fence_after();
-          const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
+          const uint32_t d_tmem = tmem_base;  // half h at column h * BN
           bool ok = true;
           for (int kb = kb0; kb < kb1; ++kb) {
             if (!gptq::mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
@@ -153,46 +156,51 @@ syrk_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_x,
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk) {
               // MN-major, 128B swizzle: MN atoms (64 elements) every 8 KB (one TMA box),
-              // 8-token K groups every 1 KB; K=16 advances 16 rows = 2 KB.
-              const uint64_t adesc = gptq::smem_desc_sw128(sa + kk * 2048, BOX_BYTES, 1024);
+              // 8-token K groups every 1 KB; K=16 advances 16 rows = 2 KB. The second half of
+              // the A tile (rows 128..255) starts two boxes further on.
               const uint64_t bdesc = gptq::smem_desc_sw128(sb + kk * 2048, BOX_BYTES, 1024);
-              gptq::mma_f16(d_tmem, adesc, bdesc, IDESC, (kb > kb0 || kk > 0) ? 1u : 0u);
+              const uint32_t acc = (kb > kb0 || kk > 0) ? 1u : 0u;
+#pragma unroll
+              for (int h = 0; h < BM / MMA_M; ++h) {
+                const uint64_t adesc = gptq::smem_desc_sw128(
+                    sa + h * 2 * BOX_BYTES + kk * 2048, BOX_BYTES, 1024);
+                gptq::mma_f16(d_tmem + (uint32_t)(h * BN), adesc, bdesc, IDESC, acc);
+              }
             }
             gptq::mma_commit(&empty[stage]);
             if (++stage == STAGES) { stage = 0; phase ^= 1; }
           }
           if (!ok) break;
-          gptq::mma_commit(&acc_full[buf]);
-          if (++buf == 2) { buf = 0; acc_phase ^= 1; }
+          gptq::mma_commit(acc_full);
+          acc_phase ^= 1;
         }
       }
     } else {
       // ------------------------------- epilogue -----------------------------------
       const int quarter = warp & 3;  // TMEM lanes 32*quarter .. 32*quarter+31
       uint8_t* my_bufs = epi_base + (warp - 2) * EPI_BUFS * EPI_TILE_BYTES;
-      int buf = 0;
       uint32_t acc_phase = 0;
       uint32_t chunk_counter = 0;
       for (long long u = blockIdx.x; u < args.n_units && !*abort_flag; u += gridDim.x) {
         const int tile = (int)(u % args.n_tiles);
         int ib, jb;
         tile_coords(tile, args.n_ib, args.n_jb, ib, jb);
-        if (!gptq::mbar_wait(&acc_full[buf], acc_phase, abort_flag)) break;
+        if (!gptq::mbar_wait(acc_full, acc_phase, abort_flag)) break;
         gptq::tc_fence_after();
-        const int row0 = ib * BM + quarter * 32;
-        const int row = row0 + lane;
-        const bool rows_live = row0 < args.d;
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int cc = 0; cc < (BM / MMA_M) * (BN / 32); ++cc) {
+          const int h = cc / (BN / 32), c = cc % (BN / 32);
+          const int row0 = ib * BM + h * MMA_M + quarter * 32;
+          const int row = row0 + lane;
           const int col0 = jb * BN + c * 32;
           uint32_t r[32];
           __syncwarp();  // tcgen05.ld is warp-collective: reconverge before every load
           const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) +
-                                 (uint32_t)(buf * BN + c * 32);
+                                 (uint32_t)(h * BN + c * 32);
           gptq::tmem_ld_32x32b_x32(taddr, r);
           gptq::tmem_ld_wait();
           // Chunk entirely below the diagonal or outside H: nothing to add.
-          const bool live = rows_live && col0 < args.d && row0 <= col0 + 31;
+          const bool live = row0 < args.d && col0 < args.d && row0 <= col0 + 31;
           if (!live) continue;
           uint8_t* sbuf = my_bufs + (chunk_counter & 1) * EPI_TILE_BYTES;
           if (chunk_counter >= 2) {
@@ -222,8 +230,8 @@ syrk_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_x,
         }
         gptq::tc_fence_before();
         __syncwarp();
-        if (lane == 0) gptq::mbar_arrive(&acc_empty[buf]);
-        if (++buf == 2) { buf = 0; acc_phase ^= 1; }
+        if (lane == 0) gptq::mbar_arrive(acc_empty);
+        acc_phase ^= 1;
       }
       if (lane == 0) gptq::bulk_wait<0>();
       __syncwarp();
@@ -271,7 +279,7 @@ int syrk_bf16_upper(float* H, int d, long long ldh, const void* X, long long n_t
   a.n_ib = (d + BM - 1) / BM;
   a.n_jb = (d + BN - 1) / BN;
   a.n_tiles = 0;
-  for (int jb = 0; jb < a.n_jb; ++jb) a.n_tiles += (2 * jb + 2 < a.n_ib) ? 2 * jb + 2 : a.n_ib;
+  for (int jb = 0; jb < a.n_jb; ++jb) a.n_tiles += (jb + 1 < a.n_ib) ? jb + 1 : a.n_ib;
   a.nkb_total = (int)((n_tokens + BK - 1) / BK);
   // The tensor core rounds toward zero when it adds into its fp32 accumulator (a one-sided
   // error of up to one ulp per step on these like-signed sums), so one accumulator covers at
