@@ -158,59 +158,81 @@ gemm_f32_small_kernel(int M, int N, int K, float alpha, const float* __restrict_
   }
 }
 
-// Staged GEMMs for short inner dimensions: one CTA per 32 x 32 output tile, 256 threads. The
-// tile's k-range (after the triangular restriction) is brought into shared memory in chunks of
-// up to 256: every thread issues all of its 16-byte loads of a chunk before storing any, so a
-// chunk costs one memory round trip. Shared memory holds both operands k-major; an operand
-// stored with k contiguous in memory is transposed on the way in, with consecutive lanes on
-// consecutive rows so that the transposing stores hit distinct banks. Each of the 8 warps then takes an eighth of the chunk for
-// the whole tile (lane: 4 rows x 8 columns, operands read as float4) and the warps' partial
-// sums are added through shared memory at the end. Needs 16-byte aligned A and B, leading
-// dimensions and K multiples of 4.
-constexpr int GT = 32, GKC = 256, GPAD = 36, G_THREADS = 256;
-constexpr int G_SMEM = 2 * GKC * GPAD * 4;  // 72 KB: As[k][m] and Bs[k][n] of one chunk
-constexpr int G_PER = GT * GKC / 4 / G_THREADS;  // 16-byte granules per thread and operand (8)
+// Staged GEMMs for short inner dimensions: one CTA per TM x 32 output tile (TM = 32 or 64),
+// 256 threads. The tile's k-range (after the triangular restriction) is brought into shared
+// memory in chunks: every thread issues all of its 16-byte loads of a chunk before storing any,
+// so a chunk costs one memory round trip, and C (when beta != 0) is fetched together with the
+// first chunk. Shared memory holds both operands k-major; an operand stored with k contiguous in
+// memory is transposed on the way in, with consecutive lanes on consecutive rows so that the
+// transposing stores hit distinct banks. The 8 warps form TM/32 groups, one per 32-row half;
+// the warps of a group split the chunk's k-range over the whole 32 x 32 half (lane: 4 rows x 8
+// columns, operands read as float4) and their partial sums are added through shared memory at
+// the end. The 64-row tile halves the CTA count of tall products so that they run in one wave.
+// Needs 16-byte aligned A and B, leading dimensions and K multiples of 4.
+constexpr int G_THREADS = 256, GPB = 36;
+template <int TM> struct Staged {
+  static constexpr int KC = TM == 32 ? 256 : 128;       // chunk length
+  static constexpr int PA = TM + 4;                     // row pitch of As[k][m]
+  static constexpr int SMEM = KC * (PA + GPB) * 4;      // 72 KB / 52 KB
+  static constexpr int PER_A = TM * KC / 4 / G_THREADS; // 16-byte granules per thread (8)
+  static constexpr int PER_B = 32 * KC / 4 / G_THREADS; // 8 / 4
+  static constexpr int GROUPS = TM / 32;
+  static constexpr int WPG = 8 / GROUPS;                // warps per 32-row group
+  static constexpr int OUT = TM * 32 / G_THREADS;       // outputs per thread in the epilogue
+};
 
+template <int TM>
 __global__ void __launch_bounds__(G_THREADS)
 gemm_f32_staged_kernel(int M, int N, int K, float alpha, const float* __restrict__ A,
                        long long lda, int transA, const float* __restrict__ B, long long ldb,
                        int transB, float beta, float* __restrict__ C, long long ldc,
                        int upper_only, int tri, const int32_t* status) {
+  using P = Staged<TM>;
   extern __shared__ __align__(16) float gsm[];
-  float* As = gsm;               // As[k][m], k relative to the chunk start
-  float* Bs = gsm + GKC * GPAD;  // Bs[k][n]
+  float* As = gsm;                   // As[k][m], k relative to the chunk start
+  float* Bs = gsm + P::KC * P::PA;   // Bs[k][n]
   if (gptq::status_bad(status)) return;
-  const int m0 = blockIdx.y * GT, n0 = blockIdx.x * GT;
-  if (upper_only && m0 > n0 + GT - 1) return;
+  const int m0 = blockIdx.y * TM, n0 = blockIdx.x * 32;
+  if (upper_only && m0 > n0 + 31) return;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int r4 = 4 * (lane >> 2), c8 = 8 * (lane & 3);
+  const int grp = warp / P::WPG, kpart = warp % P::WPG;
+  const int r4 = 32 * grp + 4 * (lane >> 2), c8 = 8 * (lane & 3);
   int k_lo, k_hi;
-  gptq_host::tri_k_range(tri, m0, n0, n0 + GT, K, k_lo, k_hi);
+  gptq_host::tri_k_range(tri, m0, n0, n0 + 32, K, k_lo, k_hi);
   k_lo &= ~3;
+
+  // C of this thread's epilogue outputs, fetched now so that its latency overlaps the operands'.
+  float cpre[P::OUT];
+#pragma unroll
+  for (int q = 0; q < P::OUT; ++q) {
+    const int e = tid + q * G_THREADS, gm = m0 + (e >> 5), gn = n0 + (e & 31);
+    cpre[q] = (beta != 0.f && gm < M && gn < N && !(upper_only && gm > gn))
+                  ? C[(long long)gm * ldc + gn] : 0.f;
+  }
+
   float acc[4][8];
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
 
-  for (int kc = k_lo; kc < k_hi; kc += GKC) {
-    const int kn = min(GKC, k_hi - kc);  // a multiple of 4
+  for (int kc = k_lo; kc < k_hi; kc += P::KC) {
+    const int kn = min(P::KC, k_hi - kc);  // a multiple of 4
     const int kq = kn >> 2;
-    float4 va[G_PER], vb[G_PER];
+    float4 va[P::PER_A], vb[P::PER_B];
     // op(A)[m0 + mm][kc + kk] and op(B)[kc + kk][n0 + nn]; granules run along the contiguous
     // direction of each operand in memory.
 #pragma unroll
-    for (int q = 0; q < G_PER; ++q) {
+    for (int q = 0; q < P::PER_A; ++q) {
       const int g = tid + q * G_THREADS;
       va[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-      vb[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (g < GT * kq) {
+      if (g < TM * kq) {
         if (!transA) {  // A[m][k]: granule = 4 consecutive k of row mm (lanes along m)
-          const int mm = g & 31, kk = 4 * (g >> 5);
+          const int mm = g % TM, kk = 4 * (g / TM);
           if (m0 + mm < M)
             va[q] = *reinterpret_cast<const float4*>(A + (long long)(m0 + mm) * lda + kc + kk);
         } else {        // A[k][m]: granule = 4 consecutive m of row kk
-          const int kk = g >> 3, mm = 4 * (g & 7);
+          const int kk = g / (TM / 4), mm = 4 * (g % (TM / 4));
           const float* src = A + (long long)(kc + kk) * lda + m0 + mm;
           if (m0 + mm + 4 <= M) {
             va[q] = *reinterpret_cast<const float4*>(src);
@@ -220,6 +242,13 @@ gemm_f32_staged_kernel(int M, int N, int K, float alpha, const float* __restrict
             if (m0 + mm + 2 < M) va[q].z = src[2];
           }
         }
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < P::PER_B; ++q) {
+      const int g = tid + q * G_THREADS;
+      vb[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (g < 32 * kq) {
         if (transB) {   // B[n][k]: granule = 4 consecutive k of row nn (lanes along n)
           const int nn = g & 31, kk = 4 * (g >> 5);
           if (n0 + nn < N)
@@ -238,37 +267,43 @@ gemm_f32_staged_kernel(int M, int N, int K, float alpha, const float* __restrict
       }
     }
 #pragma unroll
-    for (int q = 0; q < G_PER; ++q) {
+    for (int q = 0; q < P::PER_A; ++q) {
       const int g = tid + q * G_THREADS;
-      if (g < GT * kq) {
+      if (g < TM * kq) {
         if (!transA) {
-          const int mm = g & 31, kk = 4 * (g >> 5);
-          As[(kk + 0) * GPAD + mm] = va[q].x;
-          As[(kk + 1) * GPAD + mm] = va[q].y;
-          As[(kk + 2) * GPAD + mm] = va[q].z;
-          As[(kk + 3) * GPAD + mm] = va[q].w;
+          const int mm = g % TM, kk = 4 * (g / TM);
+          As[(kk + 0) * P::PA + mm] = va[q].x;
+          As[(kk + 1) * P::PA + mm] = va[q].y;
+          As[(kk + 2) * P::PA + mm] = va[q].z;
+          As[(kk + 3) * P::PA + mm] = va[q].w;
         } else {
-          *reinterpret_cast<float4*>(As + (g >> 3) * GPAD + 4 * (g & 7)) = va[q];
+          *reinterpret_cast<float4*>(As + (g / (TM / 4)) * P::PA + 4 * (g % (TM / 4))) = va[q];
         }
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < P::PER_B; ++q) {
+      const int g = tid + q * G_THREADS;
+      if (g < 32 * kq) {
         if (transB) {
           const int nn = g & 31, kk = 4 * (g >> 5);
-          Bs[(kk + 0) * GPAD + nn] = vb[q].x;
-          Bs[(kk + 1) * GPAD + nn] = vb[q].y;
-          Bs[(kk + 2) * GPAD + nn] = vb[q].z;
-          Bs[(kk + 3) * GPAD + nn] = vb[q].w;
+          Bs[(kk + 0) * GPB + nn] = vb[q].x;
+          Bs[(kk + 1) * GPB + nn] = vb[q].y;
+          Bs[(kk + 2) * GPB + nn] = vb[q].z;
+          Bs[(kk + 3) * GPB + nn] = vb[q].w;
         } else {
-          *reinterpret_cast<float4*>(Bs + (g >> 3) * GPAD + 4 * (g & 7)) = vb[q];
+          *reinterpret_cast<float4*>(Bs + (g >> 3) * GPB + 4 * (g & 7)) = vb[q];
         }
       }
     }
     __syncthreads();
-    const int kw = (kn + 7) >> 3;
-    const int kb = warp * kw, ke = min(kn, kb + kw);
+    const int kw = (kn + P::WPG - 1) / P::WPG;
+    const int kb = kpart * kw, ke = min(kn, kb + kw);
 #pragma unroll 4
     for (int k = kb; k < ke; ++k) {
-      const float4 a = *reinterpret_cast<const float4*>(As + k * GPAD + r4);
-      const float4 b0 = *reinterpret_cast<const float4*>(Bs + k * GPAD + c8);
-      const float4 b1 = *reinterpret_cast<const float4*>(Bs + k * GPAD + c8 + 4);
+      const float4 a = *reinterpret_cast<const float4*>(As + k * P::PA + r4);
+      const float4 b0 = *reinterpret_cast<const float4*>(Bs + k * GPB + c8);
+      const float4 b1 = *reinterpret_cast<const float4*>(Bs + k * GPB + c8 + 4);
       const float av[4] = {a.x, a.y, a.z, a.w};
       const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
@@ -278,24 +313,26 @@ gemm_f32_staged_kernel(int M, int N, int K, float alpha, const float* __restrict
     }
     __syncthreads();  // the next chunk (or the reduction) overwrites the staging area
   }
-  // Partial sums of the 8 warps -> shared memory (pitch 33), then 4 outputs per thread.
-  float* red = gsm;  // 8 x 32 x 33 floats, inside the staging area
+  // Partial sums of the warps -> shared memory (8 x 32 x 33 floats, inside the staging area),
+  // then each thread finishes OUT outputs by adding its group's WPG partials.
+  float* red = gsm;
+  const int rl = 4 * (lane >> 2);
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int j = 0; j < 8; ++j) red[(warp * GT + r4 + i) * 33 + c8 + j] = acc[i][j];
+    for (int j = 0; j < 8; ++j) red[(warp * 32 + rl + i) * 33 + c8 + j] = acc[i][j];
   __syncthreads();
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
+  for (int q = 0; q < P::OUT; ++q) {
     const int e = tid + q * G_THREADS, row = e >> 5, col = e & 31;
+    const int g = row >> 5, r = row & 31;
     float v = 0.f;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) v += red[(w * GT + row) * 33 + col];
+    for (int w = 0; w < P::WPG; ++w) v += red[((g * P::WPG + w) * 32 + r) * 33 + col];
     const int gm = m0 + row, gn = n0 + col;
     if (gm >= M || gn >= N || (upper_only && gm > gn)) continue;
-    float* cp = C + (long long)gm * ldc + gn;
     v *= alpha;
-    *cp = (beta == 0.f) ? v : fmaf(beta, *cp, v);
+    C[(long long)gm * ldc + gn] = (beta == 0.f) ? v : fmaf(beta, cpre[q], v);
   }
 }
 
@@ -325,12 +362,25 @@ int gemm_f32_staged(int M, int N, int K, float alpha, const float* A, long long 
                     long long ldc, bool upper_only, const int32_t* status, cudaStream_t stream,
                     int tri) {
   if (M <= 0 || N <= 0) return 0;
-  if (ensure_smem_attr(reinterpret_cast<const void*>(gemm_f32_staged_kernel), G_SMEM) != 0)
-    return GPTQ_ERR_CUDA;
-  dim3 grid((N + GT - 1) / GT, (M + GT - 1) / GT);
-  gemm_f32_staged_kernel<<<grid, G_THREADS, G_SMEM, stream>>>(
-      M, N, K, alpha, A, lda, transA ? 1 : 0, B, ldb, transB ? 1 : 0, beta, C, ldc,
-      upper_only ? 1 : 0, tri, status);
+  // 64-row tiles when 32-row ones would need more than one wave (two CTAs per SM).
+  const long long tiles32 = (long long)((N + 31) / 32) * ((M + 31) / 32);
+  if (tiles32 > 2LL * num_sms() && M >= 64) {
+    if (ensure_smem_attr(reinterpret_cast<const void*>(gemm_f32_staged_kernel<64>),
+                         Staged<64>::SMEM) != 0)
+      return GPTQ_ERR_CUDA;
+    dim3 grid((N + 31) / 32, (M + 63) / 64);
+    gemm_f32_staged_kernel<64><<<grid, G_THREADS, Staged<64>::SMEM, stream>>>(
+        M, N, K, alpha, A, lda, transA ? 1 : 0, B, ldb, transB ? 1 : 0, beta, C, ldc,
+        upper_only ? 1 : 0, tri, status);
+  } else {
+    if (ensure_smem_attr(reinterpret_cast<const void*>(gemm_f32_staged_kernel<32>),
+                         Staged<32>::SMEM) != 0)
+      return GPTQ_ERR_CUDA;
+    dim3 grid((N + 31) / 32, (M + 31) / 32);
+    gemm_f32_staged_kernel<32><<<grid, G_THREADS, Staged<32>::SMEM, stream>>>(
+        M, N, K, alpha, A, lda, transA ? 1 : 0, B, ldb, transB ? 1 : 0, beta, C, ldc,
+        upper_only ? 1 : 0, tri, status);
+  }
   return cudaGetLastError() == cudaSuccess ? 0 : GPTQ_ERR_CUDA;
 }
 

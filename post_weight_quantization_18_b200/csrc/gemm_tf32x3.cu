@@ -12,7 +12,8 @@
 // One CTA per SM (persistent), 128 x 128 output tiles, 32-wide K blocks, 3-stage ring.
 //   warp 0      TMA producer
 //   warp 1      TMEM owner + MMA issuer: per 8-wide K step three tcgen05.mma kind::tf32
-//   warps 2-5   converters: split each landed tile in place into hi and a separate lo copy
+//   warps 2-5   converters: write the lo part of each landed tile to a separate copy (the tile
+//               itself serves as hi, see below)
 //   warps 6-9   epilogue: tcgen05.ld, alpha/beta, masked stores (double-buffered accumulators)
 // Every mbarrier wait is bounded (GPTQ_ERR_TIMEOUT on expiry).
 #include "common.cuh"
@@ -220,17 +221,19 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
           uint8_t* st = smem + stage * STAGE_BYTES;
 #pragma unroll
           for (int op = 0; op < 2; ++op) {
-            float4* hi = reinterpret_cast<float4*>(st + op * 2 * TILE_BYTES);
+            const float4* hi = reinterpret_cast<const float4*>(st + op * 2 * TILE_BYTES);
             float4* lo = reinterpret_cast<float4*>(st + op * 2 * TILE_BYTES + TILE_BYTES);
 #pragma unroll 4
             for (int e = ct; e < TILE_BYTES / 16; e += N_CONV * 32) {
-              float4 x = hi[e], h, l;
-              h.x = __uint_as_float(__float_as_uint(x.x) & 0xFFFFE000u);
-              h.y = __uint_as_float(__float_as_uint(x.y) & 0xFFFFE000u);
-              h.z = __uint_as_float(__float_as_uint(x.z) & 0xFFFFE000u);
-              h.w = __uint_as_float(__float_as_uint(x.w) & 0xFFFFE000u);
-              l.x = x.x - h.x; l.y = x.y - h.y; l.z = x.z - h.z; l.w = x.w - h.w;
-              hi[e] = h;
+              // The tile stays in place as the hi operand: the tensor core reads an fp32
+              // operand of kind::tf32 as its top 19 bits, i.e. exactly x with the low 13
+              // mantissa bits cleared (results are bit-identical to storing the masked value).
+              const float4 x = hi[e];
+              float4 l;
+              l.x = x.x - __uint_as_float(__float_as_uint(x.x) & 0xFFFFE000u);
+              l.y = x.y - __uint_as_float(__float_as_uint(x.y) & 0xFFFFE000u);
+              l.z = x.z - __uint_as_float(__float_as_uint(x.z) & 0xFFFFE000u);
+              l.w = x.w - __uint_as_float(__float_as_uint(x.w) & 0xFFFFE000u);
               lo[e] = l;
             }
           }
