@@ -94,9 +94,17 @@ def _split(n):
     return m
 
 
+def _rl_launches(n):
+    """Right-looking node of nb blocks: per block a base block; below the last, the panel block
+    and the diagonal update; below the last two, the rest of the panel, the column update and
+    the trailing update; and two products of the inverse for every block but the last."""
+    nb = (n + 127) // 128
+    return nb + 2 * (nb - 1) + 3 * max(0, nb - 2) + 2 * (nb - 1)
+
+
 def _prep_launches(n):
-    if n <= 128:
-        return 1
+    if n <= 32 * 128:
+        return _rl_launches(n)
     m = _split(n)
     return 4 + _prep_launches(m) + _prep_launches(n - m)
 

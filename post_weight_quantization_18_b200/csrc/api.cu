@@ -6,8 +6,10 @@
 //  * U from H_d (gptq_prepare_hinv). With H = [[A, B], [B^T, C]] split at m:
 //        U22 = rec(C);  T = B U22^T;  S = A - T T^T;  U11 = rec(S);  U12 = -U11 (T U22)
 //    gives the upper U with H^-1 = U^T U (block form of V^-1 for H = V V^T, V upper; T is V12,
-//    S the Schur complement A - B C^-1 B^T). Blocks of <= 128 columns are factored and
-//    inverted by one CTA (prepare.cu).
+//    S the Schur complement A - B C^-1 B^T). Up to 32 blocks of 128 columns, the same
+//    factorization runs right-looking (one block column at a time, its trailing update beside
+//    the critical chain on another stream). Blocks of <= 128 columns are factored and inverted
+//    by one CTA (prepare.cu).
 //
 //  * The sweep (gptq_quantize_layer). Columns [a, b) split at m: sweep [a, m), then
 //        W[:, m:b] -= Err[:, a:m] U[a:m, m:b],
@@ -71,47 +73,200 @@ int split_point(int n) {  // a multiple of 128 near n/2, with 0 < m < n
   return m;
 }
 
-// Side streams for work off the recursion's critical path. V = T U22 of a split needs only T,
-// so it runs on a side stream while the caller's stream goes on with S and the recursion on S,
-// and the caller's stream waits for it before U12 = -U11 V. One stream and one fork/join event
-// pair per recursion depth, per device and per host thread, created on first use and kept for
-// the thread's lifetime. A thread issues its calls in order, so a pair is never in use by two
-// splits at once; event record/wait pairs are captured into CUDA graphs as dependencies.
+// Streams and events of the prepare step, per device and host thread, created on first use and
+// kept for the thread's lifetime. A thread issues its calls in order, so no stream or event is
+// used by two operations at once in a way the code below does not order explicitly; event
+// record/wait pairs are captured into CUDA graphs as dependencies.
+//  * depth[i], fork[i], join[i]: the halving recursion above the right-looking size runs
+//    V = T U22 of a split at depth i on depth[i] while the caller's stream continues.
+//  * chain / trail / inv: the three streams of the right-looking part (see rl_prepare); chain and
+//    inv have the highest priority, trail the lowest.
 constexpr int kSideDepth = 24;
 constexpr int kSideDevices = 64;
+constexpr int kRLBlocks = 32;  // right-looking nodes hold at most 32 blocks of 128 columns
 
-struct SideStreams {
+struct PrepStreams {
   bool ready = false;
-  cudaStream_t stream[kSideDepth] = {};
+  cudaStream_t depth[kSideDepth] = {};
   cudaEvent_t fork[kSideDepth] = {};
   cudaEvent_t join[kSideDepth] = {};
+  cudaStream_t chain = nullptr, trail = nullptr, inv = nullptr;
+  cudaEvent_t start = nullptr, done_chain = nullptr, done_trail = nullptr, done_inv = nullptr;
+  cudaEvent_t ev_base[kRLBlocks] = {}, ev_pd[kRLBlocks] = {}, ev_col[kRLBlocks] = {},
+              ev_trail[kRLBlocks] = {};
 };
 
-SideStreams* side_streams() {
-  thread_local SideStreams per_device[kSideDevices];
+PrepStreams* prep_streams() {
+  thread_local PrepStreams per_device[kSideDevices];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kSideDevices) return nullptr;
-  SideStreams& ss = per_device[dev];
-  if (!ss.ready) {
-    for (int i = 0; i < kSideDepth; ++i) {
-      if (cudaStreamCreateWithFlags(&ss.stream[i], cudaStreamNonBlocking) != cudaSuccess ||
-          cudaEventCreateWithFlags(&ss.fork[i], cudaEventDisableTiming) != cudaSuccess ||
-          cudaEventCreateWithFlags(&ss.join[i], cudaEventDisableTiming) != cudaSuccess)
+  PrepStreams& ps = per_device[dev];
+  if (!ps.ready) {
+    auto ev = [](cudaEvent_t* e) {
+      return cudaEventCreateWithFlags(e, cudaEventDisableTiming) == cudaSuccess;
+    };
+    int least = 0, greatest = 0;
+    if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess) return nullptr;
+    for (int i = 0; i < kSideDepth; ++i)
+      if (cudaStreamCreateWithFlags(&ps.depth[i], cudaStreamNonBlocking) != cudaSuccess ||
+          !ev(&ps.fork[i]) || !ev(&ps.join[i]))
         return nullptr;
-    }
-    ss.ready = true;
+    if (cudaStreamCreateWithPriority(&ps.chain, cudaStreamNonBlocking, greatest) != cudaSuccess ||
+        cudaStreamCreateWithPriority(&ps.inv, cudaStreamNonBlocking, greatest) != cudaSuccess ||
+        cudaStreamCreateWithPriority(&ps.trail, cudaStreamNonBlocking, least) != cudaSuccess ||
+        !ev(&ps.start) || !ev(&ps.done_chain) || !ev(&ps.done_trail) || !ev(&ps.done_inv))
+      return nullptr;
+    for (int i = 0; i < kRLBlocks; ++i)
+      if (!ev(&ps.ev_base[i]) || !ev(&ps.ev_pd[i]) || !ev(&ps.ev_col[i]) || !ev(&ps.ev_trail[i]))
+        return nullptr;
+    ps.ready = true;
   }
-  return &ss;
+  return &ps;
+}
+
+inline int ev_rec(cudaEvent_t e, cudaStream_t s) {
+  return cudaEventRecord(e, s) == cudaSuccess ? 0 : GPTQ_ERR_CUDA;
+}
+inline int ev_wait(cudaStream_t s, cudaEvent_t e) {
+  return cudaStreamWaitEvent(s, e, 0) == cudaSuccess ? 0 : GPTQ_ERR_CUDA;
+}
+
+struct InvNode {
+  int lo, mid, hi;
+};
+void inv_tree(int lo, int hi, InvNode* out, int& n) {
+  if (hi - lo < 2) return;
+  const int mid = lo + (hi - lo) / 2;
+  out[n++] = InvNode{lo, mid, hi};
+  inv_tree(lo, mid, out, n);
+  inv_tree(mid, hi, out, n);
+}
+
+// Right-looking form of the same factorization for a node [off, off+n), n <= 32 * 128: block
+// columns b = nb-1 .. 0 of 128 (block nb-1 may be shorter), A = the node's part of H.
+//   chain (critical path):   base(b): A_bb -> U_bb = V_bb^-1
+//                            Pd = A[b-1, b] U_bb^T           (V's block above the diagonal)
+//                            A[b-1, b-1] -= Pd Pd^T          (next diagonal block ready)
+//   trail (beside it):       P = A[0:b-1, b] U_bb^T          (rest of V's block column b)
+//                            A[0:b-1, b-1] -= P Pd^T         (next block column)
+//                            A[0:b-1, 0:b-1] -= P P^T        (upper; trailing update)
+//   inv:                     U = V^-1 over a balanced tree of block ranges [lo, mid, hi):
+//                            Y = V12 U22 once the right half is inverted and V's columns
+//                            mid.. are final (at level mid), U12 = -U11 Y once the left half is
+//                            inverted (at level lo). Only the U12 products of the ranges that
+//                            start at block 0 remain after the last base block.
+// V's off-diagonal blocks are held in U's upper blocks until the inverse overwrites them; Y is
+// staged in the same blocks of H, which nothing reads again by then.
+// Each wait names the level whose writes the next operation depends on.
+int rl_prepare(float* H, float* U, int d, int off, int n, PrepStreams* ps, int32_t* st,
+               cudaStream_t s) {
+  using namespace gptq_host;
+  const long long ld = d;
+  const int nb = (n + 127) / 128;
+  auto o = [&](int b) { return off + 128 * b; };
+  auto sz = [&](int b) { return (n - 128 * b) < 128 ? (n - 128 * b) : 128; };
+  auto Hp = [&](int rb, int cb) { return H + (long long)o(rb) * ld + o(cb); };
+  auto Up = [&](int rb, int cb) { return U + (long long)o(rb) * ld + o(cb); };
+  const bool conc = ps != nullptr;
+  cudaStream_t cm = conc ? ps->chain : s, ct = conc ? ps->trail : s, ci = conc ? ps->inv : s;
+  const int cap = num_sms() > 24 ? num_sms() - 16 : 0;  // persistent CTAs beside the chain
+  // Internal nodes [lo, mid, hi) of the balanced tree over the blocks (nb - 1 of them).
+  InvNode nodes[kRLBlocks];
+  int n_nodes = 0;
+  inv_tree(0, nb, nodes, n_nodes);
+  int rc = 0;
+  if (conc) {
+    if ((rc = ev_rec(ps->start, s)) || (rc = ev_wait(cm, ps->start)) ||
+        (rc = ev_wait(ct, ps->start)) || (rc = ev_wait(ci, ps->start)))
+      return rc;
+  }
+  for (int b = nb - 1; b >= 0; --b) {
+    // ---- chain ----
+    if (conc && b + 2 <= nb - 1 && (rc = ev_wait(cm, ps->ev_trail[b + 2]))) return rc;
+    if ((rc = prep_base_block(Hp(b, b), Up(b, b), sz(b), d, o(b), st, cm))) return rc;
+    if (conc && (rc = ev_rec(ps->ev_base[b], cm))) return rc;
+    if (b >= 1) {
+      if (conc && b + 1 <= nb - 1 && (rc = ev_wait(cm, ps->ev_col[b + 1]))) return rc;
+      if ((rc = gemm_f32(128, sz(b), sz(b), 1.f, Hp(b - 1, b), ld, false, Up(b, b), ld, true, 0.f,
+                         Up(b - 1, b), ld, false, st, cm, kTriBLower)))
+        return rc;
+      if (conc && (rc = ev_rec(ps->ev_pd[b], cm))) return rc;
+      if (conc && b + 1 <= nb - 1 && (rc = ev_wait(cm, ps->ev_trail[b + 1]))) return rc;
+      if ((rc = gemm_f32(128, 128, sz(b), -1.f, Up(b - 1, b), ld, false, Up(b - 1, b), ld, true,
+                         1.f, Hp(b - 1, b - 1), ld, true, st, cm)))
+        return rc;
+    }
+    // ---- trail ----
+    if (b >= 2) {
+      const int rows = 128 * (b - 1);
+      if (conc && (rc = ev_wait(ct, ps->ev_base[b]))) return rc;
+      if ((rc = gemm_f32(rows, sz(b), sz(b), 1.f, Hp(0, b), ld, false, Up(b, b), ld, true, 0.f,
+                         Up(0, b), ld, false, st, ct, kTriBLower, cap)))
+        return rc;
+      if (conc && (rc = ev_wait(ct, ps->ev_pd[b]))) return rc;
+      if ((rc = gemm_f32(rows, 128, sz(b), -1.f, Up(0, b), ld, false, Up(b - 1, b), ld, true, 1.f,
+                         Hp(0, b - 1), ld, false, st, ct, kTriNone, cap)))
+        return rc;
+      if (conc && (rc = ev_rec(ps->ev_col[b], ct))) return rc;
+      if ((rc = gemm_f32(rows, rows, sz(b), -1.f, Up(0, b), ld, false, Up(0, b), ld, true, 1.f,
+                         Hp(0, 0), ld, true, st, ct, kTriNone, cap)))
+        return rc;
+      if (conc && (rc = ev_rec(ps->ev_trail[b], ct))) return rc;
+    } else if (conc) {  // nothing to do: record so that later waits find this level's events
+      if ((rc = ev_rec(ps->ev_col[b], ct)) || (rc = ev_rec(ps->ev_trail[b], ct))) return rc;
+    }
+    // ---- inv ----
+    if (conc && (rc = ev_wait(ci, ps->ev_base[b]))) return rc;
+    // U12 = -U11 Y of the ranges that start at b, smallest first (each one's U11 is the
+    // previous one's whole range; the list is in pre-order, parents before their left
+    // children, so it is walked backwards); U12 overwrites V12, whose last readers ran at
+    // level mid.
+    for (int i = n_nodes - 1; i >= 0; --i) {
+      const InvNode& t = nodes[i];
+      if (t.lo != b) continue;
+      const int r1 = 128 * (t.mid - t.lo), r2 = n - 128 * t.mid < 128 * (t.hi - t.mid)
+                                                   ? n - 128 * t.mid : 128 * (t.hi - t.mid);
+      if (conc && (rc = ev_wait(ci, ps->ev_trail[t.mid]))) return rc;
+      if ((rc = gemm_f32(r1, r2, r1, -1.f, Up(t.lo, t.lo), ld, false, Hp(t.lo, t.mid), ld, false,
+                         0.f, Up(t.lo, t.mid), ld, false, st, ci, kTriAUpper, cap)))
+        return rc;
+    }
+    // Y = V12 U22 of the ranges split at b: U22 (the range [b, hi)) was completed just above,
+    // V's columns b.. are final after this level's panel.
+    bool waited = false;
+    for (int i = 0; i < n_nodes; ++i) {
+      const InvNode& t = nodes[i];
+      if (t.mid != b) continue;
+      const int r1 = 128 * (t.mid - t.lo), r2 = n - 128 * t.mid < 128 * (t.hi - t.mid)
+                                                   ? n - 128 * t.mid : 128 * (t.hi - t.mid);
+      if (conc && !waited) {
+        if ((rc = ev_wait(ci, ps->ev_pd[b])) || (rc = ev_wait(ci, ps->ev_col[b]))) return rc;
+        waited = true;
+      }
+      if ((rc = gemm_f32(r1, r2, r2, 1.f, Up(t.lo, t.mid), ld, false, Up(t.mid, t.mid), ld, false,
+                         0.f, Hp(t.lo, t.mid), ld, false, st, ci, kTriBUpper, cap)))
+        return rc;
+    }
+  }
+  if (conc) {
+    if ((rc = ev_rec(ps->done_chain, cm)) || (rc = ev_rec(ps->done_trail, ct)) ||
+        (rc = ev_rec(ps->done_inv, ci)) || (rc = ev_wait(s, ps->done_chain)) ||
+        (rc = ev_wait(s, ps->done_trail)) || (rc = ev_wait(s, ps->done_inv)))
+      return rc;
+  }
+  return 0;
 }
 
 // U block [off, off+n) from the damped, permuted Hessian block of the same rows/columns.
+// Nodes of at most 32 blocks use the right-looking form; larger ones split in halves:
+//   U22 = rec(C); T = B U22^T; S = A - T T^T; U11 = rec(S); U12 = -U11 (T U22).
 // The factors U22 and U11 are upper triangular with exact zeros below the diagonal, so the
 // products with them skip the k-ranges where their terms vanish.
-int rec_prepare(float* H, float* U, int d, int off, int n, int depth, SideStreams* side,
+int rec_prepare(float* H, float* U, int d, int off, int n, int depth, PrepStreams* ps,
                 int32_t* st, cudaStream_t s) {
   using namespace gptq_host;
   const long long ld = d;
-  if (n <= kPrepBase) return prep_base_block(H + off * ld + off, U + off * ld + off, n, d, off, st, s);
+  if (n <= kRLBlocks * 128) return rl_prepare(H, U, d, off, n, ps, st, s);
   const int m = split_point(n);
   const int n2 = n - m;
   float* Bblk = H + (long long)off * ld + off + m;       // H[off:off+m, off+m:off+n]
@@ -120,29 +275,27 @@ int rec_prepare(float* H, float* U, int d, int off, int n, int depth, SideStream
   float* U12 = U + (long long)off * ld + off + m;
   float* U22 = U + (long long)(off + m) * ld + off + m;
   int rc;
-  if ((rc = rec_prepare(H, U, d, off + m, n2, depth + 1, side, st, s))) return rc;
+  if ((rc = rec_prepare(H, U, d, off + m, n2, depth + 1, ps, st, s))) return rc;
   // T = B U22^T -> U12 slot (U22^T is lower triangular)
   if ((rc = gemm_f32(m, n2, n2, 1.f, Bblk, ld, false, U22, ld, true, 0.f, U12, ld, false, st, s,
                      kTriBLower)))
     return rc;
-  // V = T U22 -> B slot (B is no longer needed), on the side stream when there is one
-  const bool fork = side != nullptr && depth < kSideDepth;
+  // V = T U22 -> B slot (B is no longer needed), on the depth's stream when there is one
+  const bool fork = ps != nullptr && depth < kSideDepth;
   cudaStream_t vs = s;
   if (fork) {
-    vs = side->stream[depth];
-    if (cudaEventRecord(side->fork[depth], s) != cudaSuccess ||
-        cudaStreamWaitEvent(vs, side->fork[depth], 0) != cudaSuccess)
-      return GPTQ_ERR_CUDA;
+    vs = ps->depth[depth];
+    if ((rc = ev_rec(ps->fork[depth], s)) || (rc = ev_wait(vs, ps->fork[depth]))) return rc;
   }
   if ((rc = gemm_f32(m, n2, n2, 1.f, U12, ld, false, U22, ld, false, 0.f, Bblk, ld, false, st, vs,
                      kTriBUpper)))
     return rc;
-  if (fork && cudaEventRecord(side->join[depth], vs) != cudaSuccess) return GPTQ_ERR_CUDA;
+  if (fork && (rc = ev_rec(ps->join[depth], vs))) return rc;
   // S = A - T T^T (upper triangle) in place of A
   if ((rc = gemm_f32(m, m, n2, -1.f, U12, ld, false, U12, ld, true, 1.f, Ablk, ld, true, st, s)))
     return rc;
-  if ((rc = rec_prepare(H, U, d, off, m, depth + 1, side, st, s))) return rc;
-  if (fork && cudaStreamWaitEvent(s, side->join[depth], 0) != cudaSuccess) return GPTQ_ERR_CUDA;
+  if ((rc = rec_prepare(H, U, d, off, m, depth + 1, ps, st, s))) return rc;
+  if (fork && (rc = ev_wait(s, ps->join[depth]))) return rc;
   // U12 = -U11 V (U11 is upper triangular)
   return gemm_f32(m, n2, m, -1.f, U11, ld, false, Bblk, ld, false, 0.f, U12, ld, false, st, s,
                   kTriAUpper);
@@ -253,7 +406,7 @@ int gptq_prepare_hinv(float* H, int64_t d_in, const gptq_params* p, float* U, in
   }
   if (!rc) rc = prep_dead_damp(H, dead, d, p->percdamp, dev_status, s);
   if (!rc) rc = prep_zero_lower(U, d, s);
-  if (!rc) rc = rec_prepare(H, U, d, 0, d, 0, side_streams(), dev_status, s);
+  if (!rc) rc = rec_prepare(H, U, d, 0, d, 0, prep_streams(), dev_status, s);
   return rc ? GPTQ_ERR_CUDA : GPTQ_OK;
 }
 

@@ -403,7 +403,8 @@ namespace gptq_host {
 
 int gemm_f32(int M, int N, int K, float alpha, const float* A, long long lda, bool transA,
              const float* B, long long ldb, bool transB, float beta, float* C, long long ldc,
-             bool upper_only, const int32_t* status, cudaStream_t stream, int tri) {
+             bool upper_only, const int32_t* status, cudaStream_t stream, int tri,
+             int max_ctas) {
   if (M <= 0 || N <= 0) return 0;
   // Products up to 512 x 512 x 512 (the lower levels of the U recursion) finish sooner on
   // 32 x 32 CUDA-core tiles with the k-range staged in one round than through the tensor-core
@@ -417,7 +418,7 @@ int gemm_f32(int M, int N, int K, float alpha, const float* A, long long lda, bo
                           upper_only, status, stream, tri);
   if (gemm_tf32x3_supported(M, N, K, A, lda, B, ldb, C, ldc))
     return gemm_tf32x3(M, N, K, alpha, A, lda, transA, B, ldb, transB, beta, C, ldc, upper_only,
-                       status, stream, tri);
+                       status, stream, tri, max_ctas);
   return gemm_f32_simt(M, N, K, alpha, A, lda, transA, B, ldb, transB, beta, C, ldc, upper_only,
                        status, stream, tri);
 }

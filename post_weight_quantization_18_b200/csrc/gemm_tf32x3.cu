@@ -334,7 +334,8 @@ bool gemm_tf32x3_supported(int M, int N, int K, const float* A, long long lda, c
 // op(B) is K x N: transB=false -> B[k*ldb + n] (MN-major); transB=true -> B[n*ldb + k] (K-major).
 int gemm_tf32x3(int M, int N, int K, float alpha, const float* A, long long lda, bool transA,
                 const float* B, long long ldb, bool transB, float beta, float* C, long long ldc,
-                bool upper_only, const int32_t* status, cudaStream_t stream, int tri) {
+                bool upper_only, const int32_t* status, cudaStream_t stream, int tri,
+                int max_ctas) {
   CUtensorMap ta, tb;
   const CUtensorMapDataType f32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
   const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;               // K-major tiles
@@ -365,7 +366,8 @@ int gemm_tf32x3(int M, int N, int K, float alpha, const float* A, long long lda,
   a.status_w = const_cast<int32_t*>(status);
   if (ensure_smem_attr(reinterpret_cast<const void*>(gemm_tf32x3_kernel), SMEM_BYTES) != 0)
     return GPTQ_ERR_CUDA;
-  const int sms = num_sms();
+  int sms = num_sms();
+  if (max_ctas > 0 && max_ctas < sms) sms = max_ctas;
   const int grid = a.n_tiles < sms ? a.n_tiles : sms;
   gemm_tf32x3_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(ta, tb, a);
   return cudaGetLastError() == cudaSuccess ? 0 : GPTQ_ERR_CUDA;

@@ -32,9 +32,12 @@ __host__ __device__ inline void tri_k_range(int tri, int m0, int n0, int n_end, 
   if ((tri & kTriBUpper) && n_end < k_hi) k_hi = n_end;
 }
 
+// max_ctas > 0 caps the CTAs of the persistent tensor-core kernel (work that runs beside a
+// latency-critical chain on another stream leaves SMs free for it).
 int gemm_f32(int M, int N, int K, float alpha, const float* A, long long lda, bool transA,
              const float* B, long long ldb, bool transB, float beta, float* C, long long ldc,
-             bool upper_only, const int32_t* status, cudaStream_t stream, int tri = kTriNone);
+             bool upper_only, const int32_t* status, cudaStream_t stream, int tri = kTriNone,
+             int max_ctas = 0);
 
 int gemm_f32_simt(int M, int N, int K, float alpha, const float* A, long long lda, bool transA,
                   const float* B, long long ldb, bool transB, float beta, float* C, long long ldc,
@@ -55,7 +58,7 @@ bool gemm_tf32x3_supported(int M, int N, int K, const float* A, long long lda, c
 int gemm_tf32x3(int M, int N, int K, float alpha, const float* A, long long lda, bool transA,
                 const float* B, long long ldb, bool transB, float beta, float* C, long long ldc,
                 bool upper_only, const int32_t* status, cudaStream_t stream,
-                int tri = kTriNone);
+                int tri = kTriNone, int max_ctas = 0);
 
 // ---- prepare ----
 int prep_permute_sym(const float* H, float* Hp, const int32_t* perm, int d, cudaStream_t stream);
