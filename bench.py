@@ -96,10 +96,11 @@ def _split(n):
 
 def _rl_launches(n):
     """Right-looking node of nb blocks: per block a base block; below the last, the panel block
-    and the diagonal update; below the last two, the rest of the panel, the column update and
-    the trailing update; and two products of the inverse for every block but the last."""
+    and the diagonal update; below the last two, the rest of the panel and the trailing update
+    (with the next block column); and two products of the inverse for every block but the
+    last."""
     nb = (n + 127) // 128
-    return nb + 2 * (nb - 1) + 3 * max(0, nb - 2) + 2 * (nb - 1)
+    return nb + 2 * (nb - 1) + 2 * max(0, nb - 2) + 2 * (nb - 1)
 
 
 def _prep_launches(n):

@@ -134,9 +134,13 @@ inline int ev_wait(cudaStream_t s, cudaEvent_t e) {
 struct InvNode {
   int lo, mid, hi;
 };
+// Ranges are split in halves, except those that start at block 0: their U12 products run after
+// the last base block, so they split after at most 4 blocks and leave only products of
+// K <= 512 for the end (their large Y = V12 U22 runs while the chain finishes its last blocks).
 void inv_tree(int lo, int hi, InvNode* out, int& n) {
   if (hi - lo < 2) return;
-  const int mid = lo + (hi - lo) / 2;
+  const int half = (hi - lo) / 2;
+  const int mid = lo + (lo == 0 && half > 4 ? 4 : half);
   out[n++] = InvNode{lo, mid, hi};
   inv_tree(lo, mid, out, n);
   inv_tree(mid, hi, out, n);
@@ -148,13 +152,14 @@ void inv_tree(int lo, int hi, InvNode* out, int& n) {
 //                            Pd = A[b-1, b] U_bb^T           (V's block above the diagonal)
 //                            A[b-1, b-1] -= Pd Pd^T          (next diagonal block ready)
 //   trail (beside it):       P = A[0:b-1, b] U_bb^T          (rest of V's block column b)
-//                            A[0:b-1, b-1] -= P Pd^T         (next block column)
-//                            A[0:b-1, 0:b-1] -= P P^T        (upper; trailing update)
+//                            A[0:b-1, 0:b] -= P [P; Pd]^T    (upper; next block column and
+//                                                             trailing update)
 //   inv:                     U = V^-1 over a balanced tree of block ranges [lo, mid, hi):
 //                            Y = V12 U22 once the right half is inverted and V's columns
 //                            mid.. are final (at level mid), U12 = -U11 Y once the left half is
 //                            inverted (at level lo). Only the U12 products of the ranges that
-//                            start at block 0 remain after the last base block.
+//                            start at block 0 remain after the last base block, and the tree
+//                            keeps those small.
 // V's off-diagonal blocks are held in U's upper blocks until the inverse overwrites them; Y is
 // staged in the same blocks of H, which nothing reads again by then.
 // Each wait names the level whose writes the next operation depends on.
@@ -169,7 +174,12 @@ int rl_prepare(float* H, float* U, int d, int off, int n, PrepStreams* ps, int32
   auto Up = [&](int rb, int cb) { return U + (long long)o(rb) * ld + o(cb); };
   const bool conc = ps != nullptr;
   cudaStream_t cm = conc ? ps->chain : s, ct = conc ? ps->trail : s, ci = conc ? ps->inv : s;
-  const int cap = num_sms() > 24 ? num_sms() - 16 : 0;  // persistent CTAs beside the chain
+  // CTA budgets of the persistent GEMMs beside the chain: together they leave 16 SMs for the
+  // chain's base block and small products. Over the last few levels the trailing updates are
+  // small and the inverse runs uncapped.
+  const int sms = num_sms();
+  const int cap_inv = sms > 96 ? 24 : 0;
+  const int cap_trail = sms > 96 ? sms - 16 - cap_inv : 0;
   // Internal nodes [lo, mid, hi) of the balanced tree over the blocks (nb - 1 of them).
   InvNode nodes[kRLBlocks];
   int n_nodes = 0;
@@ -182,18 +192,20 @@ int rl_prepare(float* H, float* U, int d, int off, int n, PrepStreams* ps, int32
   }
   for (int b = nb - 1; b >= 0; --b) {
     // ---- chain ----
-    if (conc && b + 2 <= nb - 1 && (rc = ev_wait(cm, ps->ev_trail[b + 2]))) return rc;
+    // base(b) needs the trailing updates of levels b+2 and above: the chain waited for them
+    // before Pd(b+1), so one cross-stream wait per level (before Pd) covers every dependency.
     if ((rc = prep_base_block(Hp(b, b), Up(b, b), sz(b), d, o(b), st, cm))) return rc;
     if (conc && (rc = ev_rec(ps->ev_base[b], cm))) return rc;
     if (b >= 1) {
-      if (conc && b + 1 <= nb - 1 && (rc = ev_wait(cm, ps->ev_col[b + 1]))) return rc;
+      // Pd(b) reads A[b-1, b] and diag(b) writes A[b-1, b-1]; both lie in the region of the
+      // trailing update of level b+1.
+      if (conc && b + 1 <= nb - 1 && (rc = ev_wait(cm, ps->ev_trail[b + 1]))) return rc;
       if ((rc = gemm_f32(128, sz(b), sz(b), 1.f, Hp(b - 1, b), ld, false, Up(b, b), ld, true, 0.f,
-                         Up(b - 1, b), ld, false, st, cm, kTriBLower)))
+                         Up(b - 1, b), ld, false, st, cm, kTriBLower, 0, true)))
         return rc;
       if (conc && (rc = ev_rec(ps->ev_pd[b], cm))) return rc;
-      if (conc && b + 1 <= nb - 1 && (rc = ev_wait(cm, ps->ev_trail[b + 1]))) return rc;
       if ((rc = gemm_f32(128, 128, sz(b), -1.f, Up(b - 1, b), ld, false, Up(b - 1, b), ld, true,
-                         1.f, Hp(b - 1, b - 1), ld, true, st, cm)))
+                         1.f, Hp(b - 1, b - 1), ld, true, st, cm, kTriNone, 0, true)))
         return rc;
     }
     // ---- trail ----
@@ -201,17 +213,16 @@ int rl_prepare(float* H, float* U, int d, int off, int n, PrepStreams* ps, int32
       const int rows = 128 * (b - 1);
       if (conc && (rc = ev_wait(ct, ps->ev_base[b]))) return rc;
       if ((rc = gemm_f32(rows, sz(b), sz(b), 1.f, Hp(0, b), ld, false, Up(b, b), ld, true, 0.f,
-                         Up(0, b), ld, false, st, ct, kTriBLower, cap)))
+                         Up(0, b), ld, false, st, ct, kTriBLower, cap_trail)))
         return rc;
       if (conc && (rc = ev_wait(ct, ps->ev_pd[b]))) return rc;
-      if ((rc = gemm_f32(rows, 128, sz(b), -1.f, Up(0, b), ld, false, Up(b - 1, b), ld, true, 1.f,
-                         Hp(0, b - 1), ld, false, st, ct, kTriNone, cap)))
+      // A[0:b-1, 0:b] -= P [P; Pd]^T (upper): the next block column and the trailing update in
+      // one product, [P; Pd] being V's block column b, rows 0 .. b-1 (all of U[0:b, b]).
+      if ((rc = gemm_f32(rows, rows + 128, sz(b), -1.f, Up(0, b), ld, false, Up(0, b), ld, true,
+                         1.f, Hp(0, 0), ld, true, st, ct, kTriNone, cap_trail)))
         return rc;
-      if (conc && (rc = ev_rec(ps->ev_col[b], ct))) return rc;
-      if ((rc = gemm_f32(rows, rows, sz(b), -1.f, Up(0, b), ld, false, Up(0, b), ld, true, 1.f,
-                         Hp(0, 0), ld, true, st, ct, kTriNone, cap)))
+      if (conc && ((rc = ev_rec(ps->ev_col[b], ct)) || (rc = ev_rec(ps->ev_trail[b], ct))))
         return rc;
-      if (conc && (rc = ev_rec(ps->ev_trail[b], ct))) return rc;
     } else if (conc) {  // nothing to do: record so that later waits find this level's events
       if ((rc = ev_rec(ps->ev_col[b], ct)) || (rc = ev_rec(ps->ev_trail[b], ct))) return rc;
     }
@@ -228,7 +239,8 @@ int rl_prepare(float* H, float* U, int d, int off, int n, PrepStreams* ps, int32
                                                    ? n - 128 * t.mid : 128 * (t.hi - t.mid);
       if (conc && (rc = ev_wait(ci, ps->ev_trail[t.mid]))) return rc;
       if ((rc = gemm_f32(r1, r2, r1, -1.f, Up(t.lo, t.lo), ld, false, Hp(t.lo, t.mid), ld, false,
-                         0.f, Up(t.lo, t.mid), ld, false, st, ci, kTriAUpper, cap)))
+                         0.f, Up(t.lo, t.mid), ld, false, st, ci, kTriAUpper,
+                         b <= 4 ? 0 : cap_inv)))
         return rc;
     }
     // Y = V12 U22 of the ranges split at b: U22 (the range [b, hi)) was completed just above,
@@ -244,7 +256,8 @@ int rl_prepare(float* H, float* U, int d, int off, int n, PrepStreams* ps, int32
         waited = true;
       }
       if ((rc = gemm_f32(r1, r2, r2, 1.f, Up(t.lo, t.mid), ld, false, Up(t.mid, t.mid), ld, false,
-                         0.f, Hp(t.lo, t.mid), ld, false, st, ci, kTriBUpper, cap)))
+                         0.f, Hp(t.lo, t.mid), ld, false, st, ci, kTriBUpper,
+                         b <= 4 ? 0 : cap_inv)))
         return rc;
     }
   }

@@ -360,24 +360,25 @@ bool gemm_f32_staged_supported(int K, const float* A, long long lda, const float
 int gemm_f32_staged(int M, int N, int K, float alpha, const float* A, long long lda, bool transA,
                     const float* B, long long ldb, bool transB, float beta, float* C,
                     long long ldc, bool upper_only, const int32_t* status, cudaStream_t stream,
-                    int tri) {
+                    int tri, bool exclusive) {
   if (M <= 0 || N <= 0) return 0;
+  constexpr int kExclusiveSmem = 160 * 1024;  // > 227 KB - 72 KB: nothing else fits beside it
   // 64-row tiles when 32-row ones would need more than one wave (two CTAs per SM).
   const long long tiles32 = (long long)((N + 31) / 32) * ((M + 31) / 32);
   if (tiles32 > 2LL * num_sms() && M >= 64) {
-    if (ensure_smem_attr(reinterpret_cast<const void*>(gemm_f32_staged_kernel<64>),
-                         Staged<64>::SMEM) != 0)
+    const int smem = exclusive ? kExclusiveSmem : Staged<64>::SMEM;
+    if (ensure_smem_attr(reinterpret_cast<const void*>(gemm_f32_staged_kernel<64>), smem) != 0)
       return GPTQ_ERR_CUDA;
     dim3 grid((N + 31) / 32, (M + 63) / 64);
-    gemm_f32_staged_kernel<64><<<grid, G_THREADS, Staged<64>::SMEM, stream>>>(
+    gemm_f32_staged_kernel<64><<<grid, G_THREADS, smem, stream>>>(
         M, N, K, alpha, A, lda, transA ? 1 : 0, B, ldb, transB ? 1 : 0, beta, C, ldc,
         upper_only ? 1 : 0, tri, status);
   } else {
-    if (ensure_smem_attr(reinterpret_cast<const void*>(gemm_f32_staged_kernel<32>),
-                         Staged<32>::SMEM) != 0)
+    const int smem = exclusive ? kExclusiveSmem : Staged<32>::SMEM;
+    if (ensure_smem_attr(reinterpret_cast<const void*>(gemm_f32_staged_kernel<32>), smem) != 0)
       return GPTQ_ERR_CUDA;
     dim3 grid((N + 31) / 32, (M + 31) / 32);
-    gemm_f32_staged_kernel<32><<<grid, G_THREADS, Staged<32>::SMEM, stream>>>(
+    gemm_f32_staged_kernel<32><<<grid, G_THREADS, smem, stream>>>(
         M, N, K, alpha, A, lda, transA ? 1 : 0, B, ldb, transB ? 1 : 0, beta, C, ldc,
         upper_only ? 1 : 0, tri, status);
   }
@@ -404,7 +405,7 @@ namespace gptq_host {
 int gemm_f32(int M, int N, int K, float alpha, const float* A, long long lda, bool transA,
              const float* B, long long ldb, bool transB, float beta, float* C, long long ldc,
              bool upper_only, const int32_t* status, cudaStream_t stream, int tri,
-             int max_ctas) {
+             int max_ctas, bool exclusive) {
   if (M <= 0 || N <= 0) return 0;
   // Products up to 512 x 512 x 512 (the lower levels of the U recursion) finish sooner on
   // 32 x 32 CUDA-core tiles with the k-range staged in one round than through the tensor-core
@@ -412,7 +413,7 @@ int gemm_f32(int M, int N, int K, float alpha, const float* A, long long lda, bo
   // 16.3 vs 22.4); larger ones go to tcgen05 (3xTF32).
   if (K <= 512 && (long long)M * N <= 512LL * 512 && gemm_f32_staged_supported(K, A, lda, B, ldb))
     return gemm_f32_staged(M, N, K, alpha, A, lda, transA, B, ldb, transB, beta, C, ldc,
-                           upper_only, status, stream, tri);
+                           upper_only, status, stream, tri, exclusive);
   if ((long long)M * N <= 4LL * 128 * 128)
     return gemm_f32_small(M, N, K, alpha, A, lda, transA, B, ldb, transB, beta, C, ldc,
                           upper_only, status, stream, tri);

@@ -34,10 +34,13 @@ __host__ __device__ inline void tri_k_range(int tri, int m0, int n0, int n_end, 
 
 // max_ctas > 0 caps the CTAs of the persistent tensor-core kernel (work that runs beside a
 // latency-critical chain on another stream leaves SMs free for it).
+// exclusive: products on a latency-critical chain ask for enough shared memory that their CTAs
+// have their SMs to themselves (nothing launched beside them on other streams fits next to
+// them).
 int gemm_f32(int M, int N, int K, float alpha, const float* A, long long lda, bool transA,
              const float* B, long long ldb, bool transB, float beta, float* C, long long ldc,
              bool upper_only, const int32_t* status, cudaStream_t stream, int tri = kTriNone,
-             int max_ctas = 0);
+             int max_ctas = 0, bool exclusive = false);
 
 int gemm_f32_simt(int M, int N, int K, float alpha, const float* A, long long lda, bool transA,
                   const float* B, long long ldb, bool transB, float beta, float* C, long long ldc,
@@ -52,7 +55,7 @@ bool gemm_f32_staged_supported(int K, const float* A, long long lda, const float
 int gemm_f32_staged(int M, int N, int K, float alpha, const float* A, long long lda, bool transA,
                     const float* B, long long ldb, bool transB, float beta, float* C,
                     long long ldc, bool upper_only, const int32_t* status, cudaStream_t stream,
-                    int tri = kTriNone);
+                    int tri = kTriNone, bool exclusive = false);
 bool gemm_tf32x3_supported(int M, int N, int K, const float* A, long long lda, const float* B,
                            long long ldb, const float* C, long long ldc);
 int gemm_tf32x3(int M, int N, int K, float alpha, const float* A, long long lda, bool transA,

@@ -437,7 +437,11 @@ int prep_zero_lower(float* U, int d, cudaStream_t stream) {
 
 int prep_base_block(float* Hblk, float* Ublk, int n, int ld, int index0, int32_t* status,
                     cudaStream_t stream) {
-  const size_t smem = 2 * (size_t)kPrepBase * BLD * sizeof(float);
+  // The block uses 2 * 128 * 132 floats of shared memory; it asks for 180 KB so that no CTA of
+  // the products running beside it on other streams (up to 72 KB) shares its SM: the block is
+  // a single latency-bound CTA on the critical path and runs at its own speed only alone.
+  const size_t smem_used = 2 * (size_t)kPrepBase * BLD * sizeof(float);
+  const size_t smem = smem_used > 180 * 1024 ? smem_used : 180 * 1024;
   if (ensure_smem_attr(reinterpret_cast<const void*>(base_block_kernel), (int)smem) != 0)
     return GPTQ_ERR_CUDA;
   base_block_kernel<<<1, BASE_THREADS, smem, stream>>>(Hblk, Ublk, n, ld, index0, status);

@@ -53,7 +53,7 @@ def test_single_process_identity():
 
 
 def test_launch_accounting_matches_recursions():
-    """The bench's launch count follows the host recursions (d = 4096: 318 per step)."""
+    """The bench's launch count follows the host recursions (d = 4096: 288 per step)."""
     import bench
     import layer_inputs as li
-    assert bench.launches_per_step(4096, li.WORKLOADS["llama7b_attn_proj"].quant) == 318
+    assert bench.launches_per_step(4096, li.WORKLOADS["llama7b_attn_proj"].quant) == 288
