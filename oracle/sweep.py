@@ -13,6 +13,11 @@ from the current, already compensated values of those g columns of each row ([IN
 §Group Quantization gives the statistics of a run of g consecutive weights). With one scale per
 row (group_size == -1) the statistics come from the whole row at the start of the sweep.
 
+Static groups (the pre-computed group option listed among GPTQ's hyperparameters next to
+act-order): the groups are runs of g columns in the original column order, their (s, z) are
+taken once from the original (dead-column-fixed) weights before the sweep, and a column swept at
+position j uses the parameters of its original group. The routes take them as `static`.
+
 Routes
   sweep_obs       OBS update with the explicit inverse Hessian H_F^-1, downdated after every
                   column by the rank-1 formula of [GPTQ-MATH] §Recursive Inverse Hessian
@@ -27,7 +32,8 @@ Routes
                   weights are the least-squares optimum of the damped objective given the
                   already-quantized prefix. Tiny inputs only.
 
-Pinned by: the four routes agreeing (codes identical); H = I reducing to RTN; the closed-form
+Pinned by: the four routes agreeing (codes identical, also with static groups); H = I reducing
+to RTN (with static groups in any column order, the RTN of the original weights); the closed-form
 saliency Delta E_q of [GPTQ-MATH] §Minimal Error Penalty for one quantized column; invariance of
 the codes to scaling H by 4; GPTQ error <= RTN error on the small workload.
 """
@@ -38,13 +44,34 @@ import numpy as np
 from . import quantizer as qz
 
 
-class _Groups:
-    """Group bookkeeping shared by the routes (statistics over current values at group start)."""
+def static_group_params(W_orig: np.ndarray, bits: int, group_size: int, sym: bool):
+    """(S, Z) [n, G] of the runs of group_size columns of W in its original column order."""
+    n, d = W_orig.shape
+    G = (d + group_size - 1) // group_size
+    S = np.zeros((n, G))
+    Z = np.zeros((n, G))
+    for gi in range(G):
+        S[:, gi], Z[:, gi] = qz.params_from_values(
+            np.asarray(W_orig[:, gi * group_size:(gi + 1) * group_size], np.float64), bits, sym)
+    return S, Z
 
-    def __init__(self, n: int, d: int, bits: int, group_size: int, sym: bool, W0: np.ndarray):
+
+class _Groups:
+    """Group bookkeeping shared by the routes (statistics over current values at group start,
+    or fixed static parameters with a group per sweep column)."""
+
+    def __init__(self, n: int, d: int, bits: int, group_size: int, sym: bool, W0: np.ndarray,
+                 static=None):
         self.bits, self.sym = bits, sym
         self.g = d if group_size == -1 else group_size
         self.per_row = group_size == -1
+        self.gid = None
+        if static is not None:  # (S [n, G], Z [n, G], group of each sweep column [d])
+            S, Z, gid = static
+            self.S = np.array(S, np.float64, copy=True)
+            self.Z = np.array(Z, np.float64, copy=True)
+            self.gid = np.asarray(gid, np.int64)
+            return
         G = 1 if self.per_row else (d + self.g - 1) // self.g
         self.S = np.zeros((n, G))
         self.Z = np.zeros((n, G))
@@ -54,6 +81,8 @@ class _Groups:
 
     def at(self, W: np.ndarray, j: int):
         """(s, z) for column j, computing the group's statistics when j starts a group."""
+        if self.gid is not None:
+            return self.S[:, self.gid[j]], self.Z[:, self.gid[j]]
         if self.per_row:
             return self.S[:, 0], self.Z[:, 0]
         gi = j // self.g
@@ -70,7 +99,7 @@ def _quant_col(W, j, grp):
 
 
 def sweep_obs(W: np.ndarray, H_inv: np.ndarray, bits: int, group_size: int, sym: bool,
-              n_steps: int | None = None):
+              n_steps: int | None = None, static=None):
     """OBS sweep with the explicit, recursively downdated inverse Hessian.
 
     n_steps stops after that many columns (the returned W then holds the quantized prefix and
@@ -78,7 +107,7 @@ def sweep_obs(W: np.ndarray, H_inv: np.ndarray, bits: int, group_size: int, sym:
     W = np.array(W, np.float64, copy=True)
     Hi = np.array(H_inv, np.float64, copy=True)
     n, d = W.shape
-    grp = _Groups(n, d, bits, group_size, sym, W)
+    grp = _Groups(n, d, bits, group_size, sym, W, static)
     codes = np.zeros((n, d), np.uint8)
     for j in range(d if n_steps is None else n_steps):
         q, wh = _quant_col(W, j, grp)
@@ -91,11 +120,12 @@ def sweep_obs(W: np.ndarray, H_inv: np.ndarray, bits: int, group_size: int, sym:
     return codes, grp.S, grp.Z, W
 
 
-def sweep_chol(W: np.ndarray, U: np.ndarray, bits: int, group_size: int, sym: bool):
+def sweep_chol(W: np.ndarray, U: np.ndarray, bits: int, group_size: int, sym: bool,
+               static=None):
     """Unblocked sweep with rows of the upper Cholesky factor U of H^-1."""
     W = np.array(W, np.float64, copy=True)
     n, d = W.shape
-    grp = _Groups(n, d, bits, group_size, sym, W)
+    grp = _Groups(n, d, bits, group_size, sym, W, static)
     codes = np.zeros((n, d), np.uint8)
     Err = np.zeros((n, d))
     for j in range(d):
@@ -108,11 +138,11 @@ def sweep_chol(W: np.ndarray, U: np.ndarray, bits: int, group_size: int, sym: bo
 
 
 def sweep_blocked(W: np.ndarray, U: np.ndarray, bits: int, group_size: int, sym: bool,
-                  block_size: int = 128):
+                  block_size: int = 128, static=None):
     """Blocked sweep: eager updates inside each block, one lazy update of the columns after it."""
     W = np.array(W, np.float64, copy=True)
     n, d = W.shape
-    grp = _Groups(n, d, bits, group_size, sym, W)
+    grp = _Groups(n, d, bits, group_size, sym, W, static)
     codes = np.zeros((n, d), np.uint8)
     Err = np.zeros((n, d))
     for i1 in range(0, d, block_size):
@@ -128,7 +158,8 @@ def sweep_blocked(W: np.ndarray, U: np.ndarray, bits: int, group_size: int, sym:
     return codes, grp.S, grp.Z, Err
 
 
-def sweep_lstsq(W0: np.ndarray, A: np.ndarray, bits: int, group_size: int, sym: bool):
+def sweep_lstsq(W0: np.ndarray, A: np.ndarray, bits: int, group_size: int, sym: bool,
+                static=None):
     """Brute force with no inverse Hessian: A is any matrix with A^T A = H_damped (for example
     [sqrt(2) X_tm ; sqrt(lambda) I]), so the damped objective of a row is ||A (w - w0)||^2.
 
@@ -138,7 +169,7 @@ def sweep_lstsq(W0: np.ndarray, A: np.ndarray, bits: int, group_size: int, sym: 
     """
     W0 = np.array(W0, np.float64, copy=True)
     n, d = W0.shape
-    grp = _Groups(n, d, bits, group_size, sym, W0)
+    grp = _Groups(n, d, bits, group_size, sym, W0, static)
     codes = np.zeros((n, d), np.uint8)
     Wq = np.zeros((n, d))                  # dequantized prefix
     W = W0.copy()

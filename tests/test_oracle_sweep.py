@@ -134,3 +134,57 @@ def test_gptq_beats_rtn_on_small_workload(seed):
     eg = er.layer_error(W, er.dequant_matrix(L["codes"], L["S"], L["Z"], L["g_idx"]), H)
     erx = er.layer_error(W, er.dequant_matrix(R["codes"], R["S"], R["Z"], R["g_idx"]), H)
     assert eg < erx
+
+
+# ---- static groups: parameters from the original weights, groups in original column order ----
+
+@pytest.mark.parametrize("bits,gs,sym", [(4, 8, False), (3, 16, True)])
+def test_static_groups_routes_agree(bits, gs, sym):
+    """With static groups the four routes still give identical codes (act-order permutation)."""
+    W, X, H = _case(half=True, dead=(7,), seed=11)
+    P = prep.prepare(H, W, 0.01, act_order=True)
+    perm = P["perm"]
+    assert not np.array_equal(perm, np.arange(len(perm)))
+    W_orig = np.empty_like(P["W"])
+    W_orig[:, perm] = P["W"]
+    S0, Z0 = sw.static_group_params(W_orig, bits, gs, sym)
+    static = (S0, Z0, perm // gs)
+    ref = sw.sweep_obs(P["W"], P["H_inv"], bits, gs, sym, static=static)
+    c, S, Z, Err = sw.sweep_chol(P["W"], P["U"], bits, gs, sym, static=static)
+    np.testing.assert_array_equal(c, ref[0])
+    for B in (1, 8, 40):
+        np.testing.assert_array_equal(
+            sw.sweep_blocked(P["W"], P["U"], bits, gs, sym, B, static=static)[0], c)
+    lam = P["lam"]
+    A = np.vstack([np.sqrt(2.0) * X[:, perm], np.diag(np.sqrt(lam + P["dead"].astype(float)))])
+    np.testing.assert_array_equal(sw.sweep_lstsq(P["W"], A, bits, gs, sym, static=static)[0], c)
+    # the parameters are fixed before the sweep: those of the original (dead-fixed) weights
+    np.testing.assert_array_equal(S, S0)
+    np.testing.assert_array_equal(Z, Z0)
+
+
+def test_static_groups_identity_hessian_is_rtn_in_any_order():
+    """H = I with static groups: no compensation and the groups' parameters are RTN's, so the
+    codes equal RTN of the original weights whatever the column order."""
+    rng = np.random.default_rng(4)
+    W = rng.normal(0, 0.02, (12, 96))
+    R = qz.rtn(W, 4, 32, False)
+    for seed in range(3):
+        perm = np.random.default_rng(seed).permutation(96)
+        L = oracle.gptq_layer(W, np.eye(96), 4, 32, False, perm=perm, static_groups=True)
+        np.testing.assert_array_equal(L["codes"], R[0])
+        np.testing.assert_array_equal(L["S"], R[1])
+        np.testing.assert_array_equal(L["g_idx"], np.arange(96) // 32)
+
+
+def test_static_groups_differ_from_dynamic_and_keep_error_low():
+    """Static and dynamic groups are different methods (different codes); both compensate, so
+    both stay below RTN's error on a correlated layer."""
+    W, X, H = _case(n=16, d=64, N=800, seed=9)
+    Ls = oracle.gptq_layer(W, H, 4, 16, act_order=True, static_groups=True)
+    Ld = oracle.gptq_layer(W, H, 4, 16, act_order=True)
+    assert not np.array_equal(Ls["codes"], Ld["codes"])
+    R = oracle.rtn_layer(W, 4, 16)
+    def err(L):
+        return er.layer_error(W, er.dequant_matrix(L["codes"], L["S"], L["Z"], L["g_idx"]), H)
+    assert err(Ls) < err(R) and err(Ld) < err(R)
