@@ -75,6 +75,14 @@ typedef struct {
   int32_t order;      /* GPTQ_ORDER_* */
   int32_t block_size; /* lazy-update block B; must be 128 */
   float percdamp;     /* relative damping alpha: lambda = alpha * mean(diag H); 0.01 */
+  int32_t static_groups; /* 0: a group's (scale, zero) comes from its columns' current values
+                            when the sweep reaches it (groups are runs of group_size columns in
+                            sweep order). 1: groups are runs of group_size columns in the
+                            ORIGINAL order and their (scale, zero) are taken from the original
+                            weights (dead columns zero) before the sweep; with act-order each
+                            swept column uses its original group's parameters, and g_idx is
+                            c / group_size. Needs group_size > 0. Read by gptq_quantize_layer;
+                            0 when the caller zero-initialises the struct. */
 } gptq_params;
 
 /*

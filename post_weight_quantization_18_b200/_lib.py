@@ -45,13 +45,14 @@ class GPTQError(RuntimeError):
 class gptq_params(ctypes.Structure):
     _fields_ = [("bits", ctypes.c_int32), ("group_size", ctypes.c_int32), ("sym", ctypes.c_int32),
                 ("order", ctypes.c_int32), ("block_size", ctypes.c_int32),
-                ("percdamp", ctypes.c_float)]
+                ("percdamp", ctypes.c_float), ("static_groups", ctypes.c_int32)]
 
 
 def make_params(bits: int = 4, group_size: int = 128, sym: bool = False, order: int = 0,
-                block_size: int = 128, percdamp: float = 0.01) -> gptq_params:
+                block_size: int = 128, percdamp: float = 0.01,
+                static_groups: bool = False) -> gptq_params:
     return gptq_params(int(bits), int(group_size), int(bool(sym)), int(order), int(block_size),
-                       float(percdamp))
+                       float(percdamp), int(bool(static_groups)))
 
 
 def _load() -> ctypes.CDLL:

@@ -38,6 +38,8 @@ bool params_ok(const gptq_params* p) {
     return false;
   if (p->sym != 0 && p->sym != 1) return false;
   if (p->order < GPTQ_ORDER_NATURAL || p->order > GPTQ_ORDER_GIVEN) return false;
+  if (p->static_groups != 0 && p->static_groups != 1) return false;
+  if (p->static_groups && p->group_size == -1) return false;
   if (!(p->percdamp >= 0.0f) || !isfinite(p->percdamp)) return false;
   return true;
 }
@@ -46,10 +48,11 @@ struct QuantWs {
   float* Wwork;
   float* Err;
   uint8_t* codes_sweep;
+  int32_t* inv_perm;  // static groups: the inverse column permutation
   size_t bytes;
 };
 
-QuantWs quant_ws_layout(void* ws, int64_t n, int64_t d, int order) {
+QuantWs quant_ws_layout(void* ws, int64_t n, int64_t d, int order, int static_groups) {
   QuantWs w{};
   uint8_t* base = static_cast<uint8_t*>(ws);
   size_t off = 0;
@@ -61,6 +64,11 @@ QuantWs quant_ws_layout(void* ws, int64_t n, int64_t d, int order) {
   if (order != GPTQ_ORDER_NATURAL) {
     w.codes_sweep = base + off;
     off += align_up((size_t)n * d);
+  }
+  w.inv_perm = nullptr;
+  if (static_groups) {
+    w.inv_perm = reinterpret_cast<int32_t*>(base + off);
+    off += align_up((size_t)d * sizeof(int32_t));
   }
   w.bytes = off;
   return w;
@@ -322,6 +330,8 @@ struct SweepCtx {
   float* scales;
   float* zeros;
   int n, d, bits, g, sym;
+  const int32_t* perm;  // static groups: the sweep order, for each column's original group
+  int static_groups;
   int32_t* st;
   cudaStream_t s;
 };
@@ -330,7 +340,7 @@ int rec_sweep(const SweepCtx& c, int a, int b) {
   using namespace gptq_host;
   if (b - a <= 128)
     return sweep_block(c.Wwork, c.U, c.Err, c.codes, c.scales, c.zeros, c.n, c.d, a, c.bits, c.g,
-                       c.sym, c.st, c.s);
+                       c.sym, c.perm, c.static_groups, c.st, c.s);
   const int m = a + split_point(b - a);
   int rc;
   if ((rc = rec_sweep(c, a, m))) return rc;
@@ -361,7 +371,7 @@ const char* gptq_status_string(int status) {
 
 size_t gptq_workspace_size(int64_t d_out, int64_t d_in, const gptq_params* p) {
   if (!params_ok(p) || d_out < 1 || d_in < 1) return 0;
-  return quant_ws_layout(nullptr, d_out, d_in, p->order).bytes;
+  return quant_ws_layout(nullptr, d_out, d_in, p->order, p->static_groups).bytes;
 }
 
 int gptq_hessian_accumulate(float* H, int64_t d_in, int64_t ldh, const void* X, int x_dtype,
@@ -437,7 +447,7 @@ int gptq_quantize_layer(const void* W, int w_dtype, int64_t ldw, int64_t d_out, 
     return GPTQ_ERR_INVALID_ARG;
   if (w_dtype != GPTQ_BF16 && w_dtype != GPTQ_F32) return GPTQ_ERR_UNSUPPORTED;
   if (!aligned(U, 16) || !aligned(codes, 4) || !aligned(ws, 16)) return GPTQ_ERR_INVALID_ARG;
-  const QuantWs w = quant_ws_layout(ws, d_out, d_in, p->order);
+  const QuantWs w = quant_ws_layout(ws, d_out, d_in, p->order, p->static_groups);
   if (ws_bytes < w.bytes) return GPTQ_ERR_WORKSPACE;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int n = (int)d_out, d = (int)d_in;
@@ -445,13 +455,16 @@ int gptq_quantize_layer(const void* W, int w_dtype, int64_t ldw, int64_t d_out, 
   int rc = sweep_gather_w(W, w_dtype, ldw, n, d, perm, dead, w.Wwork, dev_status, s);
   if (!rc && p->group_size == -1)
     rc = sweep_row_params(w.Wwork, n, d, p->bits, p->sym, scales, zeros, dev_status, s);
+  if (!rc && p->static_groups)
+    rc = sweep_static_params(w.Wwork, perm, w.inv_perm, n, d, p->group_size, p->bits, p->sym,
+                             scales, zeros, dev_status, s);
   uint8_t* cs = (p->order == GPTQ_ORDER_NATURAL) ? codes : w.codes_sweep;
   SweepCtx c{w.Wwork, U, w.Err, cs, scales, zeros, n, d, p->bits, p->group_size, p->sym,
-             dev_status, s};
+             perm, p->static_groups, dev_status, s};
   if (!rc) rc = rec_sweep(c, 0, d);
   if (!rc && p->order != GPTQ_ORDER_NATURAL)
     rc = sweep_unpermute_codes(cs, perm, codes, n, d, dev_status, s);
-  if (!rc) rc = sweep_g_idx(perm, g_idx, d, p->group_size, s);
+  if (!rc) rc = sweep_g_idx(p->static_groups ? nullptr : perm, g_idx, d, p->group_size, s);
   return rc ? GPTQ_ERR_CUDA : GPTQ_OK;
 }
 

@@ -82,7 +82,11 @@ int sweep_row_params(const float* Wwork, int n, int d, int bits, int sym, float*
                      float* zeros, const int32_t* status, cudaStream_t stream);
 int sweep_block(float* Wwork, const float* U, float* Err, uint8_t* codes, float* scales,
                 float* zeros, int n, int d, int col0, int bits, int group_size, int sym,
-                int32_t* status, cudaStream_t stream);
+                const int32_t* perm, int static_groups, int32_t* status, cudaStream_t stream);
+// Static groups: inv = perm^-1, then (s, z) [n, d / group_size] of the original-order groups.
+int sweep_static_params(const float* Wwork, const int32_t* perm, int32_t* inv, int n, int d,
+                        int group_size, int bits, int sym, float* scales, float* zeros,
+                        const int32_t* status, cudaStream_t stream);
 int sweep_unpermute_codes(const uint8_t* codes_sweep, const int32_t* perm, uint8_t* codes, int n,
                           int d, const int32_t* status, cudaStream_t stream);
 int sweep_g_idx(const int32_t* perm, int32_t* g_idx, int d, int group_size, cudaStream_t stream);

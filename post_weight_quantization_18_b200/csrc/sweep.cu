@@ -33,6 +33,7 @@ constexpr int BLK = 128;
 constexpr int ROWS_PER_WARP = 4;
 constexpr int LANES_PER_ROW = 8;
 constexpr int SW_SMEM = BLK * BLK * 4 + BLK * 4 + 64;
+constexpr int SW_SMEM_STATIC = SW_SMEM + 3 * 16 * BLK * 4 + BLK * 4;  // + (s, 1/s, z) table
 
 // q = clamp(rne(w / s) + z, 0, maxq) with the quotient rounded as in IEEE fp32 division, but
 // formed as a multiplication by rs = 1/s (correctly rounded) wherever that cannot change the
@@ -72,14 +73,21 @@ __device__ __forceinline__ float group8_max(float v) {
   return fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
 }
 
+// STATIC: static groups (one instance each, so the default path carries no extra branch).
+template <bool STATIC>
 __global__ void __launch_bounds__(128)
 sweep_block_kernel(const __grid_constant__ CUtensorMap tmap_u, const float* __restrict__ Wwork,
                    float* __restrict__ Err, uint8_t* __restrict__ codes,
                    float* __restrict__ scales, float* __restrict__ zeros, int n, int d, int col0,
-                   int bits, int g, int sym, int32_t* status) {
+                   int bits, int g, int sym, const int32_t* __restrict__ perm,
+                   int32_t* status) {
   extern __shared__ __align__(128) float sw_smem[];
   float* Us = sw_smem;                // [128][128], zero below the diagonal
   float* invd = sw_smem + BLK * BLK;  // [128]
+  // Static groups: (s, 1/s, z) of every (row, column) of the block, [3][16][128], and the
+  // original group of each column.
+  float* stab = reinterpret_cast<float*>(sw_smem) + SW_SMEM / 4;
+  int* sgid = reinterpret_cast<int*>(stab + 3 * 16 * BLK);
   uint64_t* bar = reinterpret_cast<uint64_t*>(invd + BLK);
   __shared__ int bad;
   __shared__ volatile int abort_flag;
@@ -118,9 +126,22 @@ sweep_block_kernel(const __grid_constant__ CUtensorMap tmap_u, const float* __re
     z = zeros[rsafe];
   }
   float rs = __frcp_rn(s);
+  if (STATIC) {  // parameters fixed before the sweep, looked up per column
+    for (int t = tid; t < BLK; t += blockDim.x) sgid[t] = perm[col0 + t] / g;
+    __syncthreads();
+    for (int e = tid; e < 16 * BLK; e += blockDim.x) {
+      const int r = blockIdx.x * 16 + e / BLK;
+      const long long gi = (long long)(r < n ? r : n - 1) * G + sgid[e % BLK];
+      const float sv = scales[gi];
+      stab[e] = sv;
+      stab[16 * BLK + e] = __frcp_rn(sv);
+      stab[32 * BLK + e] = zeros[gi];
+    }
+  }
+  const int rl = warp * ROWS_PER_WARP + (lane >> 3);  // this row within the CTA
   // Group sizes divide 128 and are multiples of 4, hence powers of two: a group starts where
   // the column's low bits are zero.
-  const bool grouped = g > 0;
+  const bool grouped = g > 0 && !STATIC;
   const int gmask = grouped ? g - 1 : 0;
   const bool landed = gptq::mbar_wait(bar, 0, &abort_flag);
   if (!__syncthreads_and(landed)) {  // the copy did not arrive in time: report, touch nothing
@@ -142,7 +163,11 @@ sweep_block_kernel(const __grid_constant__ CUtensorMap tmap_u, const float* __re
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int j = 32 * c + 4 * so + e;
-        if (grouped && (j & gmask) == 0) {
+        if (STATIC) {
+          s = stab[rl * BLK + j];
+          rs = stab[16 * BLK + rl * BLK + j];
+          z = stab[32 * BLK + rl * BLK + j];
+        } else if (grouped && (j & gmask) == 0) {
           float a = sym ? 0.f : FLT_MAX, b = -FLT_MAX;
 #pragma unroll
           for (int c2 = 0; c2 < 4; ++c2)
@@ -271,10 +296,56 @@ __global__ void unpermute_codes_kernel(const uint8_t* __restrict__ cs,
   }
 }
 
+// g_idx[perm[k]] = k / g (groups in sweep order); perm == nullptr: g_idx[k] = k / g.
 __global__ void g_idx_kernel(const int32_t* __restrict__ perm, int32_t* __restrict__ g_idx, int d,
                              int g) {
   for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < d; k += gridDim.x * blockDim.x)
-    g_idx[perm[k]] = (g > 0) ? k / g : 0;
+    g_idx[perm ? perm[k] : k] = (g > 0) ? k / g : 0;
+}
+
+// inv[perm[j]] = j.
+__global__ void invert_perm_kernel(const int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+                                   int d) {
+  for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < d; j += gridDim.x * blockDim.x)
+    inv[perm[j]] = j;
+}
+
+// Static groups: (s, z) of each run of g columns in the original order, from the working copy
+// (sweep order, dead columns zero; original column c sits at sweep position inv[c]). One warp
+// per row; the lanes take the group's columns in turn.
+__global__ void static_params_kernel(const float* __restrict__ Wwork,
+                                     const int32_t* __restrict__ inv, int n, int d, int g,
+                                     int bits, int sym, float* __restrict__ scales,
+                                     float* __restrict__ zeros, const int32_t* status) {
+  if (gptq::status_bad(status)) return;
+  const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (r >= n) return;
+  const float* wr = Wwork + (long long)r * d;
+  const int G = d / g;
+  const float maxq = (float)((1 << bits) - 1);
+  for (int q = 0; q < G; ++q) {
+    float mn = FLT_MAX, mx = -FLT_MAX, am = 0.f;
+    for (int c = q * g + lane; c < q * g + g; c += 32) {
+      const float v = wr[inv[c]];
+      mn = fminf(mn, v);
+      mx = fmaxf(mx, v);
+      am = fmaxf(am, fabsf(v));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+    }
+    if (lane == 0) {
+      float sv, zv;
+      if (sym) sym_params(am, bits, sv, zv);
+      else asym_params(mn, mx, maxq, sv, zv);
+      scales[(long long)r * G + q] = sv;
+      zeros[(long long)r * G + q] = zv;
+    }
+  }
 }
 
 inline int grid_for(long long total) {
@@ -309,8 +380,9 @@ int sweep_row_params(const float* Wwork, int n, int d, int bits, int sym, float*
 
 int sweep_block(float* Wwork, const float* U, float* Err, uint8_t* codes, float* scales,
                 float* zeros, int n, int d, int col0, int bits, int group_size, int sym,
-                int32_t* status, cudaStream_t stream) {
-  if (ensure_smem_attr(reinterpret_cast<const void*>(sweep_block_kernel), SW_SMEM) != 0)
+                const int32_t* perm, int static_groups, int32_t* status, cudaStream_t stream) {
+  if (ensure_smem_attr(reinterpret_cast<const void*>(sweep_block_kernel<false>), SW_SMEM) != 0 ||
+      ensure_smem_attr(reinterpret_cast<const void*>(sweep_block_kernel<true>), SW_SMEM_STATIC) != 0)
     return GPTQ_ERR_CUDA;
   CUtensorMap tu;  // the whole U (d x d fp32), copied 128 x 128 at a time without swizzle
   if (make_tmap_2d(&tu, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, U, (uint64_t)d, (uint64_t)d,
@@ -318,8 +390,12 @@ int sweep_block(float* Wwork, const float* U, float* Err, uint8_t* codes, float*
     return GPTQ_ERR_CUDA;
   const int warps_total = (n + ROWS_PER_WARP - 1) / ROWS_PER_WARP;
   const int grid = (warps_total + 3) / 4;  // 4 warps (16 rows) per CTA
-  sweep_block_kernel<<<grid, 128, SW_SMEM, stream>>>(tu, Wwork, Err, codes, scales, zeros, n, d,
-                                                     col0, bits, group_size, sym, status);
+  if (static_groups)
+    sweep_block_kernel<true><<<grid, 128, SW_SMEM_STATIC, stream>>>(
+        tu, Wwork, Err, codes, scales, zeros, n, d, col0, bits, group_size, sym, perm, status);
+  else
+    sweep_block_kernel<false><<<grid, 128, SW_SMEM, stream>>>(
+        tu, Wwork, Err, codes, scales, zeros, n, d, col0, bits, group_size, sym, perm, status);
   return cudaGetLastError() == cudaSuccess ? 0 : GPTQ_ERR_CUDA;
 }
 
@@ -327,6 +403,16 @@ int sweep_unpermute_codes(const uint8_t* codes_sweep, const int32_t* perm, uint8
                           int d, const int32_t* status, cudaStream_t stream) {
   unpermute_codes_kernel<<<grid_for((long long)n * d), 256, 0, stream>>>(codes_sweep, perm,
                                                                          codes, n, d, status);
+  return cudaGetLastError() == cudaSuccess ? 0 : GPTQ_ERR_CUDA;
+}
+
+int sweep_static_params(const float* Wwork, const int32_t* perm, int32_t* inv, int n, int d,
+                        int group_size, int bits, int sym, float* scales, float* zeros,
+                        const int32_t* status, cudaStream_t stream) {
+  invert_perm_kernel<<<grid_for(d), 256, 0, stream>>>(perm, inv, d);
+  if (cudaGetLastError() != cudaSuccess) return GPTQ_ERR_CUDA;
+  static_params_kernel<<<(n + 7) / 8, 256, 0, stream>>>(Wwork, inv, n, d, group_size, bits, sym,
+                                                         scales, zeros, status);
   return cudaGetLastError() == cudaSuccess ? 0 : GPTQ_ERR_CUDA;
 }
 

@@ -57,15 +57,16 @@ def quantize_layer(W: torch.Tensor, X: torch.Tensor | None = None, H: torch.Tens
                    bits: int = 4, group_size: int = 128, sym: bool = False,
                    act_order: bool = False, perm: torch.Tensor | None = None,
                    percdamp: float = 0.01, prepared: tuple | None = None,
-                   check: bool = True) -> QuantizedLayer:
+                   check: bool = True, static_groups: bool = False) -> QuantizedLayer:
     """GPTQ of one linear layer. Give X (calibration activations), or H (raw 2 X^T X, clobbered),
-    or prepared = (U, perm, dead) from prepare() to share one Hessian between layers."""
+    or prepared = (U, perm, dead) from prepare() to share one Hessian between layers.
+    static_groups: groups in original column order with parameters from the original weights."""
     n, d = W.shape
     dev = W.device
     status = torch.zeros(2, dtype=torch.int32, device=dev)
     order = L.GPTQ_ORDER_GIVEN if perm is not None else (
         L.GPTQ_ORDER_DESC_ACT if act_order else L.GPTQ_ORDER_NATURAL)
-    p = L.make_params(bits, group_size, sym, order, 128, percdamp)
+    p = L.make_params(bits, group_size, sym, order, 128, percdamp, static_groups)
     ws = torch.empty(L.gptq_workspace_size(n, d, p), dtype=torch.uint8, device=dev)
     if prepared is None:
         if H is None:

@@ -25,7 +25,7 @@ def make_inputs(n, d, N, seed, x_dtype=torch.bfloat16, w_dtype=torch.bfloat16, c
 
 
 def gpu_pipeline(W, X=None, H=None, bits=4, group_size=128, sym=False, act_order=False,
-                 perm=None, percdamp=0.01):
+                 perm=None, percdamp=0.01, static_groups=False):
     """Hessian -> prepare -> sweep on the GPU. Returns host numpy arrays."""
     import post_weight_quantization_18_b200 as G
     Wd = W.cuda()
@@ -35,7 +35,8 @@ def gpu_pipeline(W, X=None, H=None, bits=4, group_size=128, sym=False, act_order
     Xd = X.cuda() if X is not None else None
     pd = torch.as_tensor(perm, dtype=torch.int32).cuda() if perm is not None else None
     out = G.quantize_layer(Wd, X=Xd, H=Hd, bits=bits, group_size=group_size, sym=sym,
-                           act_order=act_order, perm=pd, percdamp=percdamp)
+                           act_order=act_order, perm=pd, percdamp=percdamp,
+                           static_groups=static_groups)
     torch.cuda.synchronize()
     return dict(codes=out.codes.cpu().numpy(), S=out.scales.cpu().numpy().astype(np.float64),
                 Z=out.zeros.cpu().numpy().astype(np.float64),
@@ -48,7 +49,8 @@ def layer_err(W64, res, H64):
                           H64)
 
 
-def trajectory_check(W64, U64, perm, dead, codes, S, Z, bits, group_size, sym, tau=1e-3):
+def trajectory_check(W64, U64, perm, dead, codes, S, Z, bits, group_size, sym, tau=1e-3,
+                     static_groups=False):
     """Teacher-forced validity of a sweep result (tests only).
 
     Runs the column sweep in float64 with the oracle's U, but follows the decisions under test:
@@ -58,6 +60,8 @@ def trajectory_check(W64, U64, perm, dead, codes, S, Z, bits, group_size, sym, t
     recomputed from the current weights and compared with the scales/zeros under test. Several
     results are valid when a weight lies on a tie; this checks the one given without the
     cascade that a single tie decision causes in the later columns of its row.
+    With static_groups the parameters are the ones given (original group of each column), and
+    they are checked once against the statistics of the original, dead-fixed weights.
     Returns dict(bad_codes, max_excess, s_rel, z_bad).
     """
     from oracle import quantizer as qz
@@ -71,10 +75,24 @@ def trajectory_check(W64, U64, perm, dead, codes, S, Z, bits, group_size, sym, t
     excess = 0.0
     s_rel = 0.0
     z_bad = 0
+    if static_groups:
+        W_orig = np.empty_like(W)
+        W_orig[:, np.asarray(perm)] = W
+        for gi in range(d // g):
+            so, zo = qz.params_from_values(W_orig[:, gi * g:(gi + 1) * g], bits, sym)
+            s_rel = max(s_rel, float(np.max(np.abs(so - S[:, gi]) / so)))
+            if not sym:
+                mn = np.min(W_orig[:, gi * g:(gi + 1) * g], axis=1)
+                xz = -mn / S[:, gi]
+                z_bad += int(np.sum((zo != Z[:, gi]) &
+                                    (np.abs(np.abs(xz - np.floor(xz)) - 0.5) > tau)))
     for j in range(d):
         gi = 0 if group_size == -1 else j // g
+        if static_groups:
+            gi = int(perm[j]) // g
         s, z = S[:, gi], Z[:, gi]
-        if (group_size == -1 and j == 0) or (group_size != -1 and j % g == 0):
+        if not static_groups and ((group_size == -1 and j == 0) or
+                                  (group_size != -1 and j % g == 0)):
             so, zo = qz.params_from_values(W[:, j:] if group_size == -1 else W[:, j:j + g],
                                            bits, sym)
             s_rel = max(s_rel, float(np.max(np.abs(so - s) / so)))
@@ -97,7 +115,7 @@ def trajectory_check(W64, U64, perm, dead, codes, S, Z, bits, group_size, sym, t
 
 
 def compare_with_oracle(W, X, bits=4, group_size=128, sym=False, act_order=False,
-                        given_perm=False, code_agree=0.99, err_rtol=1e-3):
+                        given_perm=False, code_agree=0.99, err_rtol=1e-3, static_groups=False):
     """Full GPU pipeline vs the oracle on the same seeded inputs.
 
     Asserts: every GPU code is a valid rounding along its own trajectory (trajectory_check,
@@ -106,10 +124,12 @@ def compare_with_oracle(W, X, bits=4, group_size=128, sym=False, act_order=False
     later codes of that row, so plain agreement is a weaker, cascade-sensitive measure)."""
     W64, X64 = f64(W), f64(X)
     H64 = hs.hessian(X64)
-    ora = oracle.gptq_layer(W64, H64, bits, group_size, sym, act_order=act_order)
+    ora = oracle.gptq_layer(W64, H64, bits, group_size, sym, act_order=act_order,
+                            static_groups=static_groups)
     perm = ora["perm"] if given_perm else None
     gpu = gpu_pipeline(W, X, bits=bits, group_size=group_size, sym=sym,
-                       act_order=act_order and not given_perm, perm=perm)
+                       act_order=act_order and not given_perm, perm=perm,
+                       static_groups=static_groups)
     if act_order and not given_perm:
         assert_valid_desc_order(gpu["perm"], np.diag(H64))
     agree = float(np.mean(gpu["codes"] == ora["codes"]))
@@ -119,7 +139,7 @@ def compare_with_oracle(W, X, bits=4, group_size=128, sym=False, act_order=False
     from oracle import prepare as prep
     U64 = prep.prepare(H64, W64[:1], 0.01, perm=gpu["perm"])["U"]
     tc = trajectory_check(W64, U64, gpu["perm"], gpu["dead"], gpu["codes"], gpu["S"], gpu["Z"],
-                          bits, group_size, sym)
+                          bits, group_size, sym, static_groups=static_groups)
     msg = f"agree {agree:.6f}, rel err {rel:.2e}, trajectory {tc}"
     assert tc["bad_codes"] == 0 and tc["z_bad"] == 0, msg
     assert tc["s_rel"] <= 1e-4, msg

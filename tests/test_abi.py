@@ -45,7 +45,7 @@ def test_binding_names_match_header():
 class P(ctypes.Structure):
     _fields_ = [("bits", ctypes.c_int32), ("group_size", ctypes.c_int32), ("sym", ctypes.c_int32),
                 ("order", ctypes.c_int32), ("block_size", ctypes.c_int32),
-                ("percdamp", ctypes.c_float)]
+                ("percdamp", ctypes.c_float), ("static_groups", ctypes.c_int32)]
 
 
 def test_status_strings(lib):
@@ -62,9 +62,14 @@ def test_workspace_size(lib):
     assert lib.gptq_workspace_size(4096, 4096, ctypes.byref(ok)) == 2 * 4096 * 4096 * 4
     act = P(3, 128, 0, 1, 128, 0.01)
     assert lib.gptq_workspace_size(4096, 4096, ctypes.byref(act)) == 2 * 4096 * 4096 * 4 + 4096 * 4096
+    # static groups add the inverse column permutation (int32 per column)
+    st = P(4, 128, 0, 1, 128, 0.01, 1)
+    assert lib.gptq_workspace_size(4096, 4096, ctypes.byref(st)) == \
+        2 * 4096 * 4096 * 4 + 4096 * 4096 + 4096 * 4
     for bad in (P(5, 128, 0, 0, 128, 0.01), P(4, 96, 0, 0, 128, 0.01), P(4, 128, 0, 0, 64, 0.01),
                 P(4, 128, 2, 0, 128, 0.01), P(4, 128, 0, 3, 128, 0.01), P(4, 6, 0, 0, 128, 0.01),
-                P(4, 128, 0, 0, 128, -1.0)):
+                P(4, 128, 0, 0, 128, -1.0), P(4, -1, 1, 0, 128, 0.01, 1),
+                P(4, 128, 0, 1, 128, 0.01, 2)):
         assert lib.gptq_workspace_size(4096, 4096, ctypes.byref(bad)) == 0
     assert lib.gptq_workspace_size(0, 4096, ctypes.byref(ok)) == 0
 

@@ -106,3 +106,41 @@ def test_gptq_beats_rtn_on_gpu():
     # Expected, not a theorem ([GPTQ-MATH] §Comparison); with independent synthetic channels H is
     # nearly diagonal, where GPTQ and RTN coincide, so only a strict improvement is asserted.
     assert e_g < e_r
+
+
+# ---- static groups: original-order groups, parameters from the original weights ----
+
+def test_static_groups_act_order_given_perm_matches_oracle():
+    W, X = make_inputs(200, 512, 6000, seed=91)
+    _, _, gpu, _ = compare_with_oracle(W, X, bits=4, group_size=128, act_order=True,
+                                       given_perm=True, static_groups=True)
+    assert np.array_equal(gpu["g_idx"], np.arange(512) // 128)
+
+
+def test_static_groups_desc_act_on_gpu():
+    W, X = make_inputs(160, 384, 5000, seed=92, half_normal=True)
+    compare_with_oracle(W, X, bits=3, group_size=128, act_order=True, static_groups=True,
+                        err_rtol=5e-3)
+
+
+def test_static_groups_natural_order_g64_sym():
+    W, X = make_inputs(128, 512, 5000, seed=93)
+    compare_with_oracle(W, X, bits=4, group_size=64, sym=True, static_groups=True)
+
+
+def test_static_groups_identity_hessian_gives_rtn_in_any_order():
+    """H = I with static groups and a shuffled column order: GPU codes == GPU RTN == oracle."""
+    import post_weight_quantization_18_b200 as G
+    W, _ = make_inputs(192, 256, 8, seed=94, w_dtype=torch.float32)
+    perm = np.random.default_rng(3).permutation(256)
+    res = gpu_pipeline(W, H=np.eye(256), bits=4, group_size=64, perm=perm, static_groups=True)
+    R = oracle.rtn_layer(W.numpy(), 4, 64, False)
+    np.testing.assert_array_equal(res["codes"], R["codes"])
+    np.testing.assert_array_equal(res["g_idx"], np.arange(256) // 64)
+    p = G.make_params(4, 64)
+    codes = torch.empty((192, 256), dtype=torch.uint8, device="cuda")
+    sc = torch.empty((192, 4), device="cuda")
+    zr = torch.empty((192, 4), device="cuda")
+    G.rtn_quantize(W.cuda(), p, codes, sc, zr)
+    np.testing.assert_array_equal(res["codes"], codes.cpu().numpy())
+    np.testing.assert_array_equal(res["S"].astype(np.float32), sc.cpu().numpy())
