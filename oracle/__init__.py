@@ -29,5 +29,5 @@ in float32 with IEEE division and round-half-to-even.
 Parity status of each function is stated in its docstring ("pinned by ..."). Functions with
 no external pin say "parity unpinned".
 """
-from . import error, hessian, pack, prepare, quantizer, sweep  # noqa: F401
+from . import error, gemv, hessian, pack, prepare, quantizer, sweep  # noqa: F401
 from .layer import gptq_layer, rtn_layer  # noqa: F401
