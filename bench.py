@@ -293,6 +293,37 @@ def workload(args):
     return wl
 
 
+def measure_gemv(L, dev, hbm_gbs):
+    """Dequantizing matrix-vector product (batch 1) on a packed 8192 x 28672 int4 layer, g = 128
+    (the down projection of the 70B-shaped workload): HBM-bound. Two copies of the packed words
+    (2 x 117 MB, more than L2) are used alternately; CUDA events on the current stream."""
+    import torch
+    n, d, bits, g = 8192, 28672, 4, 128
+    ng = d // g
+    qws = [torch.randint(-2 ** 31, 2 ** 31 - 1, (n, d * bits // 32), dtype=torch.int32,
+                         device=dev) for _ in range(2)]
+    s16 = (torch.rand((n, ng), device=dev) * 0.02 + 0.001).half()
+    z16 = torch.randint(0, 2 ** bits, (n, ng), device=dev).half()
+    x = torch.randn((1, d), device=dev).half()
+    y = torch.empty((1, n), device=dev)
+    for i in range(4):
+        L.gptq_dequant_gemv(qws[i % 2], d, bits, s16, z16, g, None, x, y)
+    reps = 20
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+    torch.cuda.synchronize()
+    ev[0].record()
+    for i in range(reps):
+        L.gptq_dequant_gemv(qws[i % 2], d, bits, s16, z16, g, None, x, y)
+        ev[i + 1].record()
+    torch.cuda.synchronize()
+    us = statistics.mean(ev[i].elapsed_time(ev[i + 1]) for i in range(reps)) * 1e3
+    nbytes = n * d * bits // 8 + 2 * n * ng * 2 + d * 2 + n * 4
+    gbs = nbytes / (us * 1e-6) / 1e9
+    return {"workload": f"{n} x {d} int4 g{g}, batch 1, fp16 x, fp32 y", "us": us,
+            "bytes": nbytes, "achieved_gbs": gbs, "peak_gbs": hbm_gbs, "frac": gbs / hbm_gbs,
+            "launches": reps}
+
+
 def config_dict(args, wl, world):
     lin = wl.linears[0]
     act = wl.act(lin.act)
@@ -465,8 +496,9 @@ def run_ours(args):
     e2e_total_s = sum(e2e_ms) / 1e3
     total_s, e2e_total_s = max_over_ranks([total_s, e2e_total_s], dev)
 
+    hbm, bf16, peak_kind = peaks()
+    gemv = measure_gemv(L, dev, hbm)
     if rank == 0:
-        hbm, bf16, peak_kind = peaks()
         syrk_ms = statistics.mean(ms("syrk"))
         quant_ms = statistics.mean(ms("quant"))
         syrk_flops = float(d) * (d + 1) * N
@@ -505,6 +537,7 @@ def run_ours(args):
                          "CUDA graphs recorded from the C ABI calls, replayed",
             "clocks": clk.summary(),
             "cpu_baseline": cpu,
+            "dequant_gemv": gemv,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -237,6 +237,31 @@ int gptq_quantize_layer_noalloc(const void* W, int w_dtype, int64_t ldw, int64_t
 /* gptq_status_string — a static, human-readable name for a status code. */
 const char* gptq_status_string(int status);
 
+/*
+ * gptq_dequant_gemv — Y = X W_hat^T on the packed format: the W4A16 / W3A16 consumer of
+ * gptq_pack's output (batch 1 to 8, the low-batch decoding case).
+ *   "GPTQ: Mathematical Foundations ...", §Inference Execution and Modern Kernel Architectures:
+ *   packed codes are unpacked and dequantized, w_hat = (q - z) * s with the FP16 scale and zero,
+ *   and multiplied with FP16 activations, accumulating in higher precision.
+ *   Y[b, r] = sum_c (code[r, c] - z[r, G(c)]) * s[r, G(c)] * X[b, c], in fp32, with
+ *   G(c) = g_idx[c] or, when g_idx is NULL, c / group_size (0 when group_size == -1).
+ *
+ *   qweight     uint32 [d_out, d_in * bits / 32], the layout gptq_pack writes; 16-byte aligned
+ *   d_in        a multiple of 32; bits 2, 3, 4 or 8
+ *   scales_f16, zeros_f16  fp16 bit patterns [d_out, n_groups]
+ *   group_size  with g_idx == NULL: -1 (n_groups == 1) or a divisor of d_in
+ *               (n_groups == d_in / group_size); ignored when g_idx is given
+ *   g_idx       int32 [d_in] group of every column (values < n_groups), or NULL
+ *   X           fp16 bit patterns [batch, ldx], 16-byte aligned, ldx a multiple of 8 and >= d_in
+ *   batch       1 .. 8
+ *   Y           fp32 [batch, ldy], ldy >= d_out (written, not accumulated into)
+ * Returns GPTQ_ERR_INVALID_ARG for any other shape, alignment or parameter combination.
+ */
+int gptq_dequant_gemv(const uint32_t* qweight, int64_t d_out, int64_t d_in, int bits,
+                      const uint16_t* scales_f16, const uint16_t* zeros_f16, int64_t n_groups,
+                      int group_size, const int32_t* g_idx, const uint16_t* X, int64_t batch,
+                      int64_t ldx, float* Y, int64_t ldy, gptq_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -32,7 +32,7 @@ GPTQ_ORDER_GIVEN = 2
 
 EXPORTED = ("gptq_workspace_size", "gptq_hessian_accumulate", "gptq_prepare_hinv",
             "gptq_quantize_layer", "gptq_pack", "rtn_quantize", "gptq_status_string",
-            "gptq_quantize_layer_noalloc")
+            "gptq_quantize_layer_noalloc", "gptq_dequant_gemv")
 GPTQ_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -79,6 +79,8 @@ def _load() -> ctypes.CDLL:
     lib.gptq_pack.restype = I32
     lib.rtn_quantize.argtypes = [P, I32, I64, I64, I64, PP, P, P, P, P]
     lib.rtn_quantize.restype = I32
+    lib.gptq_dequant_gemv.argtypes = [P, I64, I64, I32, P, P, I64, I32, P, P, I64, I64, P, I64, P]
+    lib.gptq_dequant_gemv.restype = I32
     lib.gptq_status_string.argtypes = [I32]
     lib.gptq_status_string.restype = ctypes.c_char_p
     return lib
@@ -245,6 +247,29 @@ def gptq_pack(codes: torch.Tensor, bits: int, scales: torch.Tensor, zeros: torch
     rc = _lib.gptq_pack(_ptr(codes), n, d, int(bits), _ptr(scales), _ptr(zeros), G, _ptr(qweight),
                         _ptr(scales_f16), _ptr(zeros_f16), _stream())
     _check(rc, "gptq_pack")
+
+
+def gptq_dequant_gemv(qweight: torch.Tensor, d_in: int, bits: int, scales_f16: torch.Tensor,
+                      zeros_f16: torch.Tensor, group_size: int, g_idx: torch.Tensor | None,
+                      X: torch.Tensor, Y: torch.Tensor) -> None:
+    """Y [batch, d_out] (fp32) = X [batch, d_in] (fp16) @ W_hat^T from the packed layer."""
+    for t, nm in ((qweight, "qweight"), (scales_f16, "scales_f16"), (zeros_f16, "zeros_f16"),
+                  (X, "X"), (Y, "Y")):
+        _dev(t, nm)
+    if X.dtype != torch.float16 or Y.dtype != torch.float32:
+        raise ValueError("X must be float16 and Y float32")
+    if g_idx is not None:
+        _dev(g_idx, "g_idx", torch.int32, 1)
+    X2 = X.reshape(-1, X.shape[-1])
+    Y2 = Y.reshape(-1, Y.shape[-1])
+    _row_major(X2, "X")
+    _row_major(Y2, "Y")
+    n = qweight.shape[0]
+    rc = _lib.gptq_dequant_gemv(_ptr(qweight), n, int(d_in), int(bits), _ptr(scales_f16),
+                                _ptr(zeros_f16), scales_f16.shape[1], int(group_size), _ptr(g_idx),
+                                _ptr(X2), X2.shape[0], X2.stride(0), _ptr(Y2), Y2.stride(0),
+                                _stream())
+    _check(rc, "gptq_dequant_gemv")
 
 
 def rtn_quantize(W: torch.Tensor, params: gptq_params, codes: torch.Tensor, scales: torch.Tensor,

@@ -483,6 +483,34 @@ int gptq_pack(const uint8_t* codes, int64_t d_out, int64_t d_in, int bits, const
              : GPTQ_OK;
 }
 
+int gptq_dequant_gemv(const uint32_t* qweight, int64_t d_out, int64_t d_in, int bits,
+                      const uint16_t* scales_f16, const uint16_t* zeros_f16, int64_t n_groups,
+                      int group_size, const int32_t* g_idx, const uint16_t* X, int64_t batch,
+                      int64_t ldx, float* Y, int64_t ldy, gptq_stream_t stream) {
+  if (qweight == nullptr || scales_f16 == nullptr || zeros_f16 == nullptr || X == nullptr ||
+      Y == nullptr)
+    return GPTQ_ERR_INVALID_ARG;
+  if (d_out < 1 || d_in < 32 || d_in % 32 != 0 || d_in > (1 << 30) || d_out > (1 << 30))
+    return GPTQ_ERR_INVALID_ARG;
+  if (!(bits == 2 || bits == 3 || bits == 4 || bits == 8)) return GPTQ_ERR_INVALID_ARG;
+  if (batch < 1 || batch > 8 || ldx < d_in || ldx % 8 != 0 || ldy < d_out) return GPTQ_ERR_INVALID_ARG;
+  if (!aligned(qweight, 16) || !aligned(X, 16) || !aligned(scales_f16, 2) || !aligned(zeros_f16, 2))
+    return GPTQ_ERR_INVALID_ARG;
+  if (n_groups < 1 || n_groups > d_in) return GPTQ_ERR_INVALID_ARG;
+  if (g_idx == nullptr) {
+    if (group_size == -1) {
+      if (n_groups != 1) return GPTQ_ERR_INVALID_ARG;
+    } else if (group_size < 1 || d_in % group_size != 0 || n_groups != d_in / group_size) {
+      return GPTQ_ERR_INVALID_ARG;
+    }
+  }
+  return gptq_host::dequant_gemv(qweight, (int)d_out, (int)d_in, bits, scales_f16, zeros_f16,
+                                 (int)n_groups, g_idx ? 0 : group_size, g_idx, X, (int)batch, ldx,
+                                 Y, ldy, reinterpret_cast<cudaStream_t>(stream))
+             ? GPTQ_ERR_CUDA
+             : GPTQ_OK;
+}
+
 int rtn_quantize(const void* W, int w_dtype, int64_t ldw, int64_t d_out, int64_t d_in,
                  const gptq_params* p, uint8_t* codes, float* scales, float* zeros,
                  gptq_stream_t stream) {

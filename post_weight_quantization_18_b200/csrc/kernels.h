@@ -91,6 +91,12 @@ int sweep_unpermute_codes(const uint8_t* codes_sweep, const int32_t* perm, uint8
                           int d, const int32_t* status, cudaStream_t stream);
 int sweep_g_idx(const int32_t* perm, int32_t* g_idx, int d, int group_size, cudaStream_t stream);
 
+// ---- dequantizing matrix-vector product on the packed format ----
+int dequant_gemv(const uint32_t* qweight, int n, int d, int bits, const uint16_t* scales_f16,
+                 const uint16_t* zeros_f16, int n_groups, int group_size, const int32_t* g_idx,
+                 const uint16_t* x_f16, int batch, long long ldx, float* y, long long ldy,
+                 cudaStream_t stream);
+
 // ---- RTN and pack ----
 int rtn_launch(const void* W, int w_dtype, long long ldw, int n, int d, int bits, int group_size,
                int sym, uint8_t* codes, float* scales, float* zeros, cudaStream_t stream);

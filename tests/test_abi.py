@@ -25,9 +25,9 @@ def declared_functions():
 
 def test_header_declares_the_boundary():
     assert declared_functions() == sorted([
-        "gptq_hessian_accumulate", "gptq_pack", "gptq_prepare_hinv", "gptq_quantize_layer",
-        "gptq_quantize_layer_noalloc", "gptq_status_string", "gptq_workspace_size",
-        "rtn_quantize"])
+        "gptq_dequant_gemv", "gptq_hessian_accumulate", "gptq_pack", "gptq_prepare_hinv",
+        "gptq_quantize_layer", "gptq_quantize_layer_noalloc", "gptq_status_string",
+        "gptq_workspace_size", "rtn_quantize"])
 
 
 def test_every_declared_symbol_is_exported(lib):
@@ -104,3 +104,29 @@ def test_invalid_arguments_rejected_on_host(lib):
                                       ctypes.c_size_t, V, V]
     assert lib.gptq_prepare_hinv(fake, 64, ctypes.byref(p), fake, None, fake, None, 0, None,
                                  None) == 1
+
+
+def test_dequant_gemv_rejects_bad_arguments_on_host(lib):
+    V, I64 = ctypes.c_void_p, ctypes.c_int64
+    lib.gptq_dequant_gemv.argtypes = [V, I64, I64, ctypes.c_int, V, V, I64, ctypes.c_int, V, V,
+                                      I64, I64, V, I64, V]
+    fake = V(0x1000)  # 16-byte aligned, never dereferenced: every call fails its checks
+    ok = (fake, 64, 128, 4, fake, fake, 1, 128, None, fake, 1, 128, fake, 64, None)
+
+    def call(**kw):
+        names = ["q", "n", "d", "bits", "s", "z", "G", "g", "gidx", "x", "b", "ldx", "y", "ldy",
+                 "st"]
+        args = dict(zip(names, ok))
+        args.update(kw)
+        return lib.gptq_dequant_gemv(*[args[k] for k in names])
+
+    assert call(q=None) == 1
+    assert call(d=100) == 1                 # d_in not a multiple of 32
+    assert call(bits=5) == 1
+    assert call(b=0) == 1 and call(b=9) == 1
+    assert call(ldx=132) == 1               # not a multiple of 8
+    assert call(ldy=10) == 1
+    assert call(x=V(0x1004)) == 1           # X not 16-byte aligned
+    assert call(g=48) == 1                  # group size does not divide d_in
+    assert call(G=2) == 1                   # n_groups disagrees with group_size
+    assert call(g=-1, G=2) == 1
