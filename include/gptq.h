@@ -248,7 +248,8 @@ const char* gptq_status_string(int status);
  *
  *   qweight     uint32 [d_out, d_in * bits / 32], the layout gptq_pack writes; 16-byte aligned
  *   d_in        a multiple of 32; bits 2, 3, 4 or 8
- *   scales_f16, zeros_f16  fp16 bit patterns [d_out, n_groups]
+ *   scales_f16, zeros_f16  fp16 bit patterns [d_out, n_groups]; zero points are integers in
+ *               [0, 2^bits), as gptq_pack stores them (other values are rounded to an integer)
  *   group_size  with g_idx == NULL: -1 (n_groups == 1) or a divisor of d_in
  *               (n_groups == d_in / group_size); ignored when g_idx is given
  *   g_idx       int32 [d_in] group of every column (values < n_groups), or NULL

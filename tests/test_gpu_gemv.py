@@ -62,6 +62,13 @@ def _w_hat(qn, sn, zn, gi, d, bits):
     (256, 1024, 2, -1, False, 2),     # one group per row
     (384, 2048, 8, 32, False, 8),     # 8-bit, batch 8
     (300, 1024, 4, 16, False, 1),     # groups shorter than a 32-column run
+    # tensor-core path: groups of whole 128-column chunks, d_in a multiple of 128
+    (1000, 4096, 4, 256, False, 3),   # ragged last 16-row tile, groups over two chunks
+    (70, 128, 4, 128, False, 1),      # one chunk per row, fewer chunks than warps
+    (384, 2048, 8, 128, False, 8),    # 8-bit, full batch
+    (136, 3072, 2, 128, False, 5),    # 2-bit, odd batch
+    (64, 1152, 4, -1, False, 1),      # one group per row, chunk count not a multiple of warps
+    (96, 1056, 4, -1, False, 2),      # d_in not a multiple of 128: warp-per-row path
 ])
 def test_dequant_gemv_matches_oracle(n, d, bits, g, perm, batch):
     qw, s16, z16, g_idx, _ = _packed_layer(n, d, bits, g, seed=n + d + bits, gidx_perm=perm)
