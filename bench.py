@@ -294,9 +294,10 @@ def workload(args):
 
 
 def measure_gemv(L, dev, hbm_gbs):
-    """Dequantizing matrix-vector product (batch 1) on a packed 8192 x 28672 int4 layer, g = 128
-    (the down projection of the 70B-shaped workload): HBM-bound. Two copies of the packed words
-    (2 x 117 MB, more than L2) are used alternately; CUDA events on the current stream."""
+    """Dequantizing matrix-vector product on a packed 8192 x 28672 int4 layer, g = 128 (the down
+    projection of the 70B-shaped workload), batch 1 (the reported figure) and batch 8: HBM-bound.
+    Two copies of the packed words (2 x 117 MB, more than L2) are used alternately; CUDA events
+    on the current stream."""
     import torch
     n, d, bits, g = 8192, 28672, 4, 128
     ng = d // g
@@ -304,24 +305,31 @@ def measure_gemv(L, dev, hbm_gbs):
                          device=dev) for _ in range(2)]
     s16 = (torch.rand((n, ng), device=dev) * 0.02 + 0.001).half()
     z16 = torch.randint(0, 2 ** bits, (n, ng), device=dev).half()
-    x = torch.randn((1, d), device=dev).half()
-    y = torch.empty((1, n), device=dev)
-    for i in range(4):
-        L.gptq_dequant_gemv(qws[i % 2], d, bits, s16, z16, g, None, x, y)
     reps = 20
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
-    torch.cuda.synchronize()
-    ev[0].record()
-    for i in range(reps):
-        L.gptq_dequant_gemv(qws[i % 2], d, bits, s16, z16, g, None, x, y)
-        ev[i + 1].record()
-    torch.cuda.synchronize()
-    us = statistics.mean(ev[i].elapsed_time(ev[i + 1]) for i in range(reps)) * 1e3
-    nbytes = n * d * bits // 8 + 2 * n * ng * 2 + d * 2 + n * 4
+
+    def timed(batch):
+        x = torch.randn((batch, d), device=dev).half()
+        y = torch.empty((batch, n), device=dev)
+        for i in range(4):
+            L.gptq_dequant_gemv(qws[i % 2], d, bits, s16, z16, g, None, x, y)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+        torch.cuda.synchronize()
+        ev[0].record()
+        for i in range(reps):
+            L.gptq_dequant_gemv(qws[i % 2], d, bits, s16, z16, g, None, x, y)
+            ev[i + 1].record()
+        torch.cuda.synchronize()
+        us = statistics.mean(ev[i].elapsed_time(ev[i + 1]) for i in range(reps)) * 1e3
+        nbytes = n * d * bits // 8 + 2 * n * ng * 2 + batch * (d * 2 + n * 4)
+        return us, nbytes
+
+    us, nbytes = timed(1)
+    us8, nbytes8 = timed(8)
     gbs = nbytes / (us * 1e-6) / 1e9
     return {"workload": f"{n} x {d} int4 g{g}, batch 1, fp16 x, fp32 y", "us": us,
             "bytes": nbytes, "achieved_gbs": gbs, "peak_gbs": hbm_gbs, "frac": gbs / hbm_gbs,
-            "launches": reps}
+            "batch8_us": us8, "batch8_gbs": nbytes8 / (us8 * 1e-6) / 1e9,
+            "launches": 2 * (reps + 4)}
 
 
 def config_dict(args, wl, world):
