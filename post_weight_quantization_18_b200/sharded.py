@@ -3,9 +3,9 @@
 The method shards with a single exchange:
 
 * Tokens. H = 2 X^T X is a sum over calibration tokens ("GPTQ: Mathematical Foundations ...",
-  §Second-Order Taylor Expansion; "INT4 GPTQ", §The Quantization Error and Layerwise Objective),
-  so each rank forms the upper triangle of its own tokens' sum with gptq_hessian_accumulate
-  and one all-reduce (sum) over the group gives every rank the whole H.
+  §Second-Order Taylor Expansion; "INT4 and GPTQ Quantization", §The Quantization Error and
+  Layerwise Objective), so each rank forms the upper triangle of its own tokens' sum with
+  gptq_hessian_accumulate and one all-reduce (sum) over the group gives every rank the whole H.
 * Prepare. Replicated: every rank runs gptq_prepare_hinv on the same bits of H, and the
   kernels are deterministic, so every rank holds the same U, permutation and dead columns.
 * Rows. Given U, the column sweep treats the rows of W independently (each row's error only
