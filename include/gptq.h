@@ -7,6 +7,8 @@
  *   gptq_quantize_layer      column sweep with OBS compensation and lazy block updates
  *   gptq_pack                codes -> packed int words, scales/zeros -> fp16
  *   rtn_quantize             round-to-nearest baseline with the same quantizer
+ *   gptq_dequant_gemv        Y = X W_hat^T on the packed layer (batch 1 to 8), the format's consumer
+ *   gptq_quantize_layer_noalloc  gptq_quantize_layer on a fixed device scratch array
  *
  * Sources (page title, section):
  *   [INT4-GPTQ] "INT4 and GPTQ Quantization" (beta.fermi.ai wiki)
