@@ -271,10 +271,13 @@ def run_reference(args):
     value = lin.d_out * lin.d_in / per
     sample = (f"each step: FP64 oracle H on {tok_sample} of {act.n_tokens} tokens (scaled), full "
               f"{act.d}x{act.d} prepare, blocked sweep of {row_sample} of {lin.d_out} rows (scaled)")
-    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 0,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": config_dict(args, wl, world=1),
+    # Same line as this bench's own arm (n_gpus and config of the launch); what actually ran,
+    # the oracle on this host's cores, is described under cpu_baseline.
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": per * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_dict(args, wl, world=args.gpus),
             "cpu_baseline": {"kind": "oracle", "value": value, "unit": UNIT, "cores": cpu_cores(),
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
