@@ -144,3 +144,35 @@ def test_static_groups_identity_hessian_gives_rtn_in_any_order():
     G.rtn_quantize(W.cuda(), p, codes, sc, zr)
     np.testing.assert_array_equal(res["codes"], codes.cpu().numpy())
     np.testing.assert_array_equal(res["S"].astype(np.float32), sc.cpu().numpy())
+
+
+def _with_degenerate_rows(W):
+    """An all-zero row, a constant row, and a row whose first group is zero and whose second is
+    constant (values exact in bf16). The zero group comes first on purpose: after a constant
+    group that the symmetric quantizer reproduces almost exactly, a zero group would hold only
+    the rounding noise of that group's errors (about 1e-9 in fp32, 1e-17 in fp64), and its codes
+    would be decided by that noise on either side."""
+    W = W.clone()
+    W[0] = 0.0
+    W[1] = 0.03125
+    W[2, :128] = 0.0
+    W[2, 128:256] = -0.0625
+    return W
+
+
+@pytest.mark.parametrize("g,sym", [(128, False), (128, True), (-1, False)])
+def test_degenerate_rows_and_groups(g, sym):
+    """Constant and all-zero ranges take s = 1 on both sides: RTN bit for bit, and the GPTQ layer
+    stays a valid rounding trajectory that matches the oracle."""
+    import post_weight_quantization_18_b200 as G
+    W, X = make_inputs(64, 512, 3000, seed=321)
+    W = _with_degenerate_rows(W)
+    codes, s, z = G.rtn(W.cuda(), 4, g, sym)
+    ora = oracle.rtn_layer(W.float().numpy(), 4, g, sym)
+    np.testing.assert_array_equal(codes.cpu().numpy(), ora["codes"])
+    np.testing.assert_array_equal(s.cpu().numpy(), ora["S"])
+    np.testing.assert_array_equal(z.cpu().numpy(), ora["Z"])
+    assert np.all(ora["S"][0] == 1.0)
+    if not sym:
+        assert np.all(ora["S"][1] == 1.0)
+    compare_with_oracle(W, X, bits=4, group_size=g, sym=sym)
