@@ -1,10 +1,17 @@
-// gemm_f32.cu — C = alpha * op(A) op(B) + beta * C in fp32 (row-major), CUDA-core version.
+// gemm_f32.cu — C = alpha * op(A) op(B) + beta * C in fp32 (row-major) on CUDA cores, and the
+// dispatcher gemm_f32() that routes every fp32 product of the library.
 //
 // Serves the fp32 pieces of the path: the lazy trailing update W[:, F] -= Err_B U[B, F]
 // ("GPTQ: Mathematical Foundations ...", §2 Lazy Batch Updates), the GEMM steps of the
-// Cholesky / triangular-inverse recursion, and the Hessian of fp32 calibration inputs.
-// 128x128 output tile per 256-thread CTA, 8x8 outputs per thread, k-slabs of 16 staged in
-// shared memory (transposes resolved while staging).
+// Cholesky / triangular-inverse schedule, and the Hessian of fp32 calibration inputs.
+//   gemm_f32_staged_kernel  products up to 512 x 512 x 512 (the critical chain of prepare and
+//                           the sweep's small updates): 32 x 32 (or 64 x 32) output tile per
+//                           CTA, the tile's whole k-range staged with one round of 16-byte
+//                           loads, split over the warps, partial sums added in shared memory.
+//   gemm_f32_small_kernel   other small outputs (up to 4 tiles of 128 x 128).
+//   gemm_f32_simt_kernel    operands TMA cannot address: 128 x 128 tile per 256-thread CTA,
+//                           8 x 8 outputs per thread, k-slabs of 16 staged in shared memory.
+// Everything else goes to the tcgen05 3xTF32 kernel (gemm_tf32x3.cu).
 #include "common.cuh"
 #include "kernels.h"
 

@@ -10,9 +10,10 @@
 //
 // U is obtained without forming H^-1: factor H_d = V V^T with V upper triangular (Cholesky
 // from the last column), then U = V^-1. (V^-T V^-1 = H_d^-1 and V^-1 is upper with a positive
-// diagonal, so it is the unique upper Cholesky factor of H_d^-1.) The host recursion in
-// api.cu splits the matrix into halves and uses GEMMs; the base blocks of at most 128 columns
-// are factored and inverted here by one CTA in shared memory.
+// diagonal, so it is the unique upper Cholesky factor of H_d^-1.) The host schedule in api.cu
+// runs right-looking over 128-column blocks up to 4096 columns (splitting larger matrices in
+// halves first) and does the off-diagonal work with GEMMs; each 128-column diagonal block is
+// factored and inverted here by one CTA in shared memory.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -120,10 +121,10 @@ __global__ void zero_lower_kernel(float* U, int d) {
 }
 
 // Base block (n <= 128): the damped block H_d (upper triangle, leading dimension ld) -> the
-// U block = V^-1 where H_d = V V^T, V upper. The same recursion as the host one, inside one CTA
-// of 16 warps on two shared-memory matrices (A: the block being factored, U: the result):
-//   128 -> 64 -> 32 -> 16-column leaves. Each split does the four block products of the host
-//   recursion on the tensor cores (warp-level m16n8k8 TF32 with the three-term hi/lo split, so
+// U block = V^-1 where H_d = V V^T, V upper. A recursion on halves (the one the host uses above
+// 4096 columns), inside one CTA of 16 warps on two shared-memory matrices (A: the block being
+// factored, U: the result): 128 -> 64 -> 32 -> 16-column leaves. Each split does its four
+//   block products on the tensor cores (warp-level m16n8k8 TF32 with the three-term hi/lo split, so
 //   the products carry fp32 accuracy), skipping the k-ranges where the triangular operand is
 //   zero and computing only the upper tiles of the symmetric update. A 32-column node (two
 //   leaves and its four 16 x 16 products) runs on one warp without block barriers; a leaf is
