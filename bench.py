@@ -13,6 +13,9 @@ ABI. Default workload: Llama-7B attention projection, W 4096 x 4096 bf16, X 2621
 Prints one JSON line (rank 0). Under torchrun each rank quantizes its own layer (independent
 problems, no collective on the data path: weak scaling); the timed duration is the max over ranks.
 --impl reference times the FP64 CPU oracle on bounded samples of the same workload.
+Outside the timed steps the line also reports the per-stage times (breakdown_ms), the SYRK
+roofline, the end-to-end rate from pinned host buffers (e2e), the oracle's rate (cpu_baseline),
+and the dequantizing GEMV on a packed 8192 x 28672 int4 layer (dequant_gemv).
 """
 from __future__ import annotations
 
