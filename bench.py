@@ -537,6 +537,8 @@ def run_ours(args):
             "breakdown_ms": {"hessian_syrk": syrk_ms, "prepare": statistics.mean(ms("prep")),
                              "quantize_sweep": quant_ms, "pack": statistics.mean(ms("pack"))},
             "syrk_tflops": syrk_tflops,
+            # the same time counted as the full 2 d^2 N product (upper and lower triangle)
+            "syrk_tflops_2d2n_equivalent": 2.0 * d * d * N / (syrk_ms * 1e-3) / 1e12,
             "sweep_gbs": sweep_bytes / (quant_ms * 1e-3) / 1e9,
             "roofline": {"bound": "tensor", "kernel": "syrk_bf16_tcgen05_kernel",
                          "achieved": syrk_tflops, "peak": bf16, "unit": "TFLOP/s",
