@@ -9,7 +9,7 @@
 // Architectures: eight 4-bit weights per int32; "INT4 and GPTQ Quantization", §Group
 // Quantization: scale and zero in FP16): each row is an LSB-first bit stream, code k at bits
 // [b*k, b*k + b); word w holds stream bits [32w, 32w + 32). One thread packs 32 codes, which
-// fill exactly b words.
+// fill exactly b words (pack32.cuh); rows of whole chunks take vector loads and stores.
 #include <float.h>
 
 #include <cuda_bf16.h>
@@ -17,6 +17,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "pack32.cuh"
 
 namespace {
 
@@ -101,6 +102,36 @@ __global__ void pack_kernel(const uint8_t* __restrict__ codes, int n, int d, int
   }
 }
 
+// Fast path for rows of whole 32-code chunks: one thread per chunk, the 32 codes in two 16-byte
+// loads and the words in one 16-byte store (4 and 8 bits: two for 8), one 8-byte store (2 bits)
+// or three word stores (3 bits). The host takes it only when codes is 16-byte aligned, d is a
+// multiple of 32 and qweight is aligned for the store width, so every access is aligned.
+template <int BITS>
+__global__ void pack_vec_kernel(const uint8_t* __restrict__ codes, int n, int d,
+                                uint32_t* __restrict__ qweight) {
+  const long long item = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (item >= (long long)n * (d / 32)) return;
+  const uint8_t* src;
+  uint32_t* out;
+  gptq::pack_chunk_ptrs<BITS>(codes, qweight, d, item, src, out);
+  const uint4 a = __ldg(reinterpret_cast<const uint4*>(src));
+  const uint4 b = __ldg(reinterpret_cast<const uint4*>(src) + 1);
+  const uint32_t c[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  uint32_t w[BITS];
+  gptq::pack32<BITS>(c, w);
+  if constexpr (BITS == 4) {
+    *reinterpret_cast<uint4*>(out) = make_uint4(w[0], w[1], w[2], w[3]);
+  } else if constexpr (BITS == 8) {
+    reinterpret_cast<uint4*>(out)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    reinterpret_cast<uint4*>(out)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  } else if constexpr (BITS == 2) {
+    *reinterpret_cast<uint2*>(out) = make_uint2(w[0], w[1]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < BITS; ++i) out[i] = w[i];
+  }
+}
+
 __global__ void to_f16_kernel(const float* __restrict__ a, const float* __restrict__ b,
                               uint16_t* __restrict__ ah, uint16_t* __restrict__ bh,
                               long long count) {
@@ -138,7 +169,20 @@ int pack_launch(const uint8_t* codes, int n, int d, int bits, const float* scale
                 const float* zeros, long long n_groups, uint32_t* qweight, uint16_t* scales_f16,
                 uint16_t* zeros_f16, cudaStream_t stream) {
   const long long items = (long long)n * ((d + 31) / 32);
-  pack_kernel<<<(unsigned)((items + 255) / 256), 256, 0, stream>>>(codes, n, d, bits, qweight);
+  const unsigned blocks = (unsigned)((items + 255) / 256);
+  const int store_align = bits == 2 ? 8 : (bits == 3 ? 4 : 16);
+  const bool vec = d % 32 == 0 && (reinterpret_cast<uintptr_t>(codes) & 15) == 0 &&
+                   (reinterpret_cast<uintptr_t>(qweight) & (uintptr_t)(store_align - 1)) == 0;
+  if (vec && bits == 2)
+    pack_vec_kernel<2><<<blocks, 256, 0, stream>>>(codes, n, d, qweight);
+  else if (vec && bits == 3)
+    pack_vec_kernel<3><<<blocks, 256, 0, stream>>>(codes, n, d, qweight);
+  else if (vec && bits == 4)
+    pack_vec_kernel<4><<<blocks, 256, 0, stream>>>(codes, n, d, qweight);
+  else if (vec && bits == 8)
+    pack_vec_kernel<8><<<blocks, 256, 0, stream>>>(codes, n, d, qweight);
+  else
+    pack_kernel<<<blocks, 256, 0, stream>>>(codes, n, d, bits, qweight);
   if (cudaGetLastError() != cudaSuccess) return GPTQ_ERR_CUDA;
   const long long cnt = (long long)n * n_groups;
   to_f16_kernel<<<grid_cap((cnt + 255) / 256), 256, 0, stream>>>(scales, zeros, scales_f16,
