@@ -25,6 +25,7 @@
 #include <cuda_bf16.h>
 
 #include "common.cuh"
+#include "gather4.cuh"
 #include "kernels.h"
 
 namespace {
@@ -232,24 +233,23 @@ sweep_block_kernel(const __grid_constant__ CUtensorMap tmap_u, const float* __re
   if (!finite && live) gptq::set_status(status, GPTQ_ERR_NONFINITE, col0);
 }
 
-// Wwork[r][k] = dead[k] ? 0 : W[r][perm[k]] as fp32 (bf16 widened exactly).
-template <typename T>
+// Wwork[r][k] = dead[k] ? 0 : W[r][perm[k]] as fp32 (bf16 widened exactly). A thread owns four
+// consecutive columns (d is a multiple of 128): their sources and liveness are read once, then
+// for each of its rows (blockIdx.y, grid-stride) four loads and one 16-byte store.
+template <typename T>  // float, or uint16_t holding bf16 bit patterns
 __global__ void gather_w_kernel(const T* __restrict__ W, long long ldw, int n, int d,
                                 const int32_t* __restrict__ perm, const uint8_t* __restrict__ dead,
                                 float* __restrict__ Wwork, const int32_t* status) {
   if (gptq::status_bad(status)) return;
-  const long long total = (long long)n * d;
-  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
-       e += (long long)gridDim.x * blockDim.x) {
-    const int r = (int)(e / d), k = (int)(e % d);
-    float v = 0.f;
-    if (!dead[k]) {
-      if constexpr (sizeof(T) == 2)
-        v = __bfloat162float(W[(long long)r * ldw + perm[k]]);
-      else
-        v = W[(long long)r * ldw + perm[k]];
-    }
-    Wwork[e] = v;
+  const int k0 = 4 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (k0 >= d) return;
+  int32_t src[4];
+  bool live[4];
+  gptq::gather4_cols(perm, dead, k0, src, live);
+  for (long long r = blockIdx.y; r < n; r += gridDim.y) {
+    float v[4];
+    gptq::gather4_row<T>(W, ldw, r, src, live, v);
+    *reinterpret_cast<float4*>(Wwork + r * d + k0) = make_float4(v[0], v[1], v[2], v[3]);
   }
 }
 
@@ -361,13 +361,15 @@ namespace gptq_host {
 int sweep_gather_w(const void* W, int w_dtype, long long ldw, int n, int d, const int32_t* perm,
                    const uint8_t* dead, float* Wwork, const int32_t* status,
                    cudaStream_t stream) {
-  const int gr = grid_for((long long)n * d);
+  // d is a multiple of 128 and Wwork 16-byte aligned (checked by the entry point), so every
+  // thread's four columns exist and its float4 store is aligned.
+  const dim3 grid((unsigned)((d / 4 + 255) / 256), (unsigned)(n < 65535 ? n : 65535));
   if (w_dtype == GPTQ_BF16)
-    gather_w_kernel<__nv_bfloat16><<<gr, 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(W), ldw, n, d, perm, dead, Wwork, status);
+    gather_w_kernel<uint16_t><<<grid, 256, 0, stream>>>(static_cast<const uint16_t*>(W), ldw, n,
+                                                        d, perm, dead, Wwork, status);
   else
-    gather_w_kernel<float><<<gr, 256, 0, stream>>>(static_cast<const float*>(W), ldw, n, d, perm,
-                                                   dead, Wwork, status);
+    gather_w_kernel<float><<<grid, 256, 0, stream>>>(static_cast<const float*>(W), ldw, n, d,
+                                                     perm, dead, Wwork, status);
   return cudaGetLastError() == cudaSuccess ? 0 : GPTQ_ERR_CUDA;
 }
 

@@ -46,3 +46,39 @@ def test_pack_fast_path_code_on_cpu_matches_oracle(tmp_path, bits, d):
     assert r.returncode == 0, r.stderr
     words = np.frombuffer((tmp_path / "words.bin").read_bytes(), np.uint32).reshape(n, -1)
     np.testing.assert_array_equal(words, pk.pack_rows(codes, bits))
+
+
+@pytest.mark.skipif(shutil.which("g++") is None, reason="needs g++")
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("n,d,ldw", [(5, 128, 128), (3, 1152, 1200), (70000, 128, 130)])
+def test_w_gather_code_on_cpu(tmp_path, dtype, n, d, ldw):
+    """The per-thread code of the sweep's W gather (gather4.cuh, the functions gather_w_kernel
+    calls), run on the CPU over the host's launch grid (including more rows than grid.y), gives
+    W[:, perm] widened to fp32 with the dead columns zeroed."""
+    import numpy as np
+    import torch
+    exe = tmp_path / "gather4_check"
+    r = subprocess.run(["g++", "-std=c++17", "-O2", "-Wall", "-Werror", "-Wno-unknown-pragmas",
+                        "-I", os.path.join(ROOT, "post_weight_quantization_18_b200", "csrc"),
+                        os.path.join(ROOT, "tests", "c", "gather4_check.cpp"), "-o", str(exe)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    rng = np.random.default_rng(n + d)
+    W = torch.from_numpy(rng.standard_normal((n, ldw)).astype(np.float32))
+    if dtype == "bf16":
+        W = W.to(torch.bfloat16)
+        raw = W.view(torch.int16).numpy().tobytes()
+    else:
+        raw = W.numpy().tobytes()
+    perm = rng.permutation(d).astype(np.int32)
+    dead = (rng.random(d) < 0.1).astype(np.uint8)
+    for name, data in (("w.bin", raw), ("perm.bin", perm.tobytes()), ("dead.bin", dead.tobytes())):
+        (tmp_path / name).write_bytes(data)
+    r = subprocess.run([str(exe), dtype, str(n), str(d), str(ldw)] +
+                       [str(tmp_path / x) for x in ("w.bin", "perm.bin", "dead.bin", "out.bin")],
+                       capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stderr
+    got = np.frombuffer((tmp_path / "out.bin").read_bytes(), np.float32).reshape(n, d)
+    want = W.float().numpy()[:, :d][:, perm].copy()
+    want[:, dead.astype(bool)] = 0.0
+    np.testing.assert_array_equal(got, want)
