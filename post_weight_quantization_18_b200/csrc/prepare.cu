@@ -16,6 +16,7 @@
 // factored and inverted here by one CTA in shared memory.
 #include "common.cuh"
 #include "kernels.h"
+#include "tri_fill.cuh"
 
 namespace {
 
@@ -111,12 +112,15 @@ __global__ void dead_damp_kernel(float* __restrict__ H, uint8_t* __restrict__ de
   for (int j = threadIdx.x; j < d; j += blockDim.x) H[(long long)j * d + j] += lam;
 }
 
+// U's strictly lower triangle = 0: rows on grid y, columns strided over grid x (tri_fill.cuh).
 __global__ void zero_lower_kernel(float* U, int d) {
-  const long long total = (long long)d * d;
-  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
-       e += (long long)gridDim.x * blockDim.x) {
-    const int a = (int)(e / d), b = (int)(e % d);
-    if (a > b) U[e] = 0.f;
+  for (long long r = blockIdx.y; r < d; r += gridDim.y) {
+    long long lo, hi;
+    gptq::tri_row_span(gptq::kStrictLower, r, d, lo, hi);
+    float* row = U + r * d;
+    for (long long c = lo + blockIdx.x * (long long)blockDim.x + threadIdx.x; c < hi;
+         c += (long long)gridDim.x * blockDim.x)
+      row[c] = 0.f;
   }
 }
 
@@ -432,7 +436,8 @@ int prep_dead_damp(float* H, uint8_t* dead, int d, float percdamp, int32_t* stat
 }
 
 int prep_zero_lower(float* U, int d, cudaStream_t stream) {
-  zero_lower_kernel<<<grid_for((long long)d * d), 256, 0, stream>>>(U, d);
+  const dim3 grid((unsigned)((d + 1023) / 1024), (unsigned)(d < 65535 ? d : 65535));
+  zero_lower_kernel<<<grid, 256, 0, stream>>>(U, d);
   return cudaGetLastError() == cudaSuccess ? 0 : GPTQ_ERR_CUDA;
 }
 

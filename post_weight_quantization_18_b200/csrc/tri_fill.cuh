@@ -1,0 +1,29 @@
+// tri_fill.cuh — which elements of a row-major square matrix a triangle-clearing launch
+// writes. Rows go to the grid's y dimension (grid-stride), and the threads of the x dimension
+// stride along the row's span. No per-element division: the row is known and the span is
+// contiguous. Host-and-device code, so that the kernels' index arithmetic is also checked on
+// the CPU.
+#pragma once
+
+#if defined(__CUDACC__)
+#define GPTQ_HD __host__ __device__ __forceinline__
+#else
+#define GPTQ_HD inline
+#endif
+
+namespace gptq {
+
+enum TriPart { kStrictLower = 0, kUpperWithDiag = 1 };
+
+// Columns [lo, hi) of row r that belong to the part.
+GPTQ_HD void tri_row_span(int part, long long r, int d, long long& lo, long long& hi) {
+  if (part == kStrictLower) {
+    lo = 0;
+    hi = r < d ? r : d;
+  } else {
+    lo = r;
+    hi = d;
+  }
+}
+
+}  // namespace gptq

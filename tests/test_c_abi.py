@@ -82,3 +82,28 @@ def test_w_gather_code_on_cpu(tmp_path, dtype, n, d, ldw):
     want = W.float().numpy()[:, :d][:, perm].copy()
     want[:, dead.astype(bool)] = 0.0
     np.testing.assert_array_equal(got, want)
+
+
+@pytest.mark.skipif(shutil.which("g++") is None, reason="needs g++")
+@pytest.mark.parametrize("part,d,ld", [(0, 1, 1), (0, 37, 37), (0, 1500, 1500), (1, 37, 40),
+                                       (1, 1500, 1504)])
+def test_triangle_clear_index_math_on_cpu(tmp_path, part, d, ld):
+    """The triangle-clearing kernels' index arithmetic (tri_fill.cuh) over the host's launch grid
+    clears exactly the strictly lower triangle (part 0) or the upper triangle with the diagonal
+    (part 1, padded rows left alone) and nothing else."""
+    import numpy as np
+    exe = tmp_path / "tri_fill_check"
+    r = subprocess.run(["g++", "-std=c++17", "-O2", "-Wall", "-Werror",
+                        "-I", os.path.join(ROOT, "post_weight_quantization_18_b200", "csrc"),
+                        os.path.join(ROOT, "tests", "c", "tri_fill_check.cpp"), "-o", str(exe)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe), str(part), str(d), str(ld)], capture_output=True, text=True,
+                       timeout=120)
+    assert r.returncode == 0, r.stderr
+    got = np.array([[c == "1" for c in line] for line in r.stdout.split()], dtype=bool)
+    want = np.ones((d, ld), bool)
+    rows, cols = np.indices((d, d))
+    cleared = rows > cols if part == 0 else rows <= cols
+    want[:, :d][cleared] = False
+    np.testing.assert_array_equal(got, want)
