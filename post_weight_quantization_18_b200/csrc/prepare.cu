@@ -20,26 +20,28 @@
 
 namespace {
 
-// Hp[a][b] = H[pi a][pi b] on the upper triangle, reading H's upper triangle symmetrically.
+// Hp[a][b] = H[pi a][pi b] on the upper triangle, reading H's upper triangle symmetrically:
+// rows on grid y, columns of the row's span strided over grid x (tri_fill.cuh).
 __global__ void permute_sym_kernel(const float* __restrict__ H, float* __restrict__ Hp,
                                    const int32_t* __restrict__ perm, int d) {
-  const long long total = (long long)d * d;
-  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
-       e += (long long)gridDim.x * blockDim.x) {
-    const int a = (int)(e / d), b = (int)(e % d);
-    if (a > b) continue;
-    const int i = perm[a], j = perm[b];
-    const int lo = i < j ? i : j, hi = i < j ? j : i;
-    Hp[(long long)a * d + b] = H[(long long)lo * d + hi];
+  for (long long a = blockIdx.y; a < d; a += gridDim.y) {
+    long long lo, hi;
+    gptq::tri_row_span(gptq::kUpperWithDiag, a, d, lo, hi);
+    const int pa = perm[a];
+    for (long long b = lo + blockIdx.x * (long long)blockDim.x + threadIdx.x; b < hi;
+         b += (long long)gridDim.x * blockDim.x)
+      gptq::permute_sym_elem(H, Hp, perm, d, a, pa, b);
   }
 }
 
+// dst's upper triangle (with the diagonal) = src's, same layout.
 __global__ void copy_upper_kernel(const float* __restrict__ src, float* __restrict__ dst, int d) {
-  const long long total = (long long)d * d;
-  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
-       e += (long long)gridDim.x * blockDim.x) {
-    const int a = (int)(e / d), b = (int)(e % d);
-    if (a <= b) dst[e] = src[e];
+  for (long long a = blockIdx.y; a < d; a += gridDim.y) {
+    long long lo, hi;
+    gptq::tri_row_span(gptq::kUpperWithDiag, a, d, lo, hi);
+    for (long long b = lo + blockIdx.x * (long long)blockDim.x + threadIdx.x; b < hi;
+         b += (long long)gridDim.x * blockDim.x)
+      dst[a * d + b] = src[a * d + b];
   }
 }
 
@@ -410,12 +412,14 @@ inline int grid_for(long long total) {
 namespace gptq_host {
 
 int prep_permute_sym(const float* H, float* Hp, const int32_t* perm, int d, cudaStream_t stream) {
-  permute_sym_kernel<<<grid_for((long long)d * d), 256, 0, stream>>>(H, Hp, perm, d);
+  const dim3 grid((unsigned)((d + 1023) / 1024), (unsigned)(d < 65535 ? d : 65535));
+  permute_sym_kernel<<<grid, 256, 0, stream>>>(H, Hp, perm, d);
   return cudaGetLastError() == cudaSuccess ? 0 : GPTQ_ERR_CUDA;
 }
 
 int prep_copy_upper(const float* src, float* dst, int d, cudaStream_t stream) {
-  copy_upper_kernel<<<grid_for((long long)d * d), 256, 0, stream>>>(src, dst, d);
+  const dim3 grid((unsigned)((d + 1023) / 1024), (unsigned)(d < 65535 ? d : 65535));
+  copy_upper_kernel<<<grid, 256, 0, stream>>>(src, dst, d);
   return cudaGetLastError() == cudaSuccess ? 0 : GPTQ_ERR_CUDA;
 }
 

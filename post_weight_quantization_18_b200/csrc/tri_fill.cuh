@@ -26,4 +26,13 @@ GPTQ_HD void tri_row_span(int part, long long r, int d, long long& lo, long long
   }
 }
 
+// Element (a, b), b >= a, of the permuted Hessian's upper triangle: Hp[a][b] = H[pi a][pi b],
+// read from H's upper triangle (H symmetric, only i <= j stored). pa = perm[a].
+GPTQ_HD void permute_sym_elem(const float* H, float* Hp, const int* perm, int d, long long a,
+                              int pa, long long b) {
+  const int j = perm[b];
+  const long long lo = pa < j ? pa : j, hi = pa < j ? j : pa;
+  Hp[a * d + b] = H[lo * d + hi];
+}
+
 }  // namespace gptq

@@ -107,3 +107,32 @@ def test_triangle_clear_index_math_on_cpu(tmp_path, part, d, ld):
     cleared = rows > cols if part == 0 else rows <= cols
     want[:, :d][cleared] = False
     np.testing.assert_array_equal(got, want)
+
+
+@pytest.mark.skipif(shutil.which("g++") is None, reason="needs g++")
+@pytest.mark.parametrize("d", [1, 37, 1100])
+def test_permute_sym_index_math_on_cpu(tmp_path, d):
+    """The act-order permutation of H (permute_sym_kernel's loops over the host's launch grid,
+    tri_fill.cuh) writes exactly Hp[a][b] = H[pi a][pi b] on the upper triangle, reading only
+    H's upper triangle, and nothing below the diagonal."""
+    import numpy as np
+    exe = tmp_path / "permute_sym_check"
+    r = subprocess.run(["g++", "-std=c++17", "-O2", "-Wall", "-Werror",
+                        "-I", os.path.join(ROOT, "post_weight_quantization_18_b200", "csrc"),
+                        os.path.join(ROOT, "tests", "c", "permute_sym_check.cpp"), "-o", str(exe)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    rng = np.random.default_rng(d)
+    S = rng.standard_normal((d, d)).astype(np.float32)
+    S = S + S.T
+    H = np.triu(S) + np.tril(np.full((d, d), np.nan, np.float32), -1)   # lower part never read
+    perm = rng.permutation(d).astype(np.int32)
+    (tmp_path / "h.bin").write_bytes(H.tobytes())
+    (tmp_path / "perm.bin").write_bytes(perm.tobytes())
+    r = subprocess.run([str(exe), str(d), str(tmp_path / "h.bin"), str(tmp_path / "perm.bin"),
+                        str(tmp_path / "out.bin")], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stderr
+    got = np.frombuffer((tmp_path / "out.bin").read_bytes(), np.float32).reshape(d, d)
+    iu = np.triu_indices(d)
+    np.testing.assert_array_equal(got[iu], S[perm][:, perm][iu])
+    assert np.all(got[np.tril_indices(d, -1)] == -1.0)
