@@ -27,6 +27,7 @@
 #include "common.cuh"
 #include "gather4.cuh"
 #include "kernels.h"
+#include "tri_fill.cuh"
 
 namespace {
 
@@ -288,11 +289,13 @@ __global__ void unpermute_codes_kernel(const uint8_t* __restrict__ cs,
                                        uint8_t* __restrict__ codes, int n, int d,
                                        const int32_t* status) {
   if (gptq::status_bad(status)) return;
-  const long long total = (long long)n * d;
-  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
-       e += (long long)gridDim.x * blockDim.x) {
-    const int r = (int)(e / d), k = (int)(e % d);
-    codes[(long long)r * d + perm[k]] = cs[e];
+  // Rows on grid y, columns strided over grid x (tri_fill.cuh): no per-element division.
+  for (long long r = blockIdx.y; r < n; r += gridDim.y) {
+    long long lo, hi;
+    gptq::tri_row_span(gptq::kWholeRow, r, d, lo, hi);
+    for (long long k = lo + blockIdx.x * (long long)blockDim.x + threadIdx.x; k < hi;
+         k += (long long)gridDim.x * blockDim.x)
+      gptq::unpermute_elem(cs, perm, codes, d, r, k);
   }
 }
 
@@ -403,8 +406,8 @@ int sweep_block(float* Wwork, const float* U, float* Err, uint8_t* codes, float*
 
 int sweep_unpermute_codes(const uint8_t* codes_sweep, const int32_t* perm, uint8_t* codes, int n,
                           int d, const int32_t* status, cudaStream_t stream) {
-  unpermute_codes_kernel<<<grid_for((long long)n * d), 256, 0, stream>>>(codes_sweep, perm,
-                                                                         codes, n, d, status);
+  const dim3 grid((unsigned)((d + 1023) / 1024), (unsigned)(n < 65535 ? n : 65535));
+  unpermute_codes_kernel<<<grid, 256, 0, stream>>>(codes_sweep, perm, codes, n, d, status);
   return cudaGetLastError() == cudaSuccess ? 0 : GPTQ_ERR_CUDA;
 }
 

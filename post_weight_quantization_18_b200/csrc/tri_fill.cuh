@@ -13,17 +13,26 @@
 
 namespace gptq {
 
-enum TriPart { kStrictLower = 0, kUpperWithDiag = 1 };
+enum TriPart { kStrictLower = 0, kUpperWithDiag = 1, kWholeRow = 2 };
 
 // Columns [lo, hi) of row r that belong to the part.
 GPTQ_HD void tri_row_span(int part, long long r, int d, long long& lo, long long& hi) {
   if (part == kStrictLower) {
     lo = 0;
     hi = r < d ? r : d;
-  } else {
+  } else if (part == kUpperWithDiag) {
     lo = r;
     hi = d;
+  } else {
+    lo = 0;
+    hi = d;
   }
+}
+
+// Codes back in the original column order: codes[r][perm[k]] = cs[r][k] (rows of d codes).
+GPTQ_HD void unpermute_elem(const unsigned char* cs, const int* perm, unsigned char* codes, int d,
+                            long long r, long long k) {
+  codes[r * d + perm[k]] = cs[r * d + k];
 }
 
 // Element (a, b), b >= a, of the permuted Hessian's upper triangle: Hp[a][b] = H[pi a][pi b],

@@ -136,3 +136,30 @@ def test_permute_sym_index_math_on_cpu(tmp_path, d):
     iu = np.triu_indices(d)
     np.testing.assert_array_equal(got[iu], S[perm][:, perm][iu])
     assert np.all(got[np.tril_indices(d, -1)] == -1.0)
+
+
+@pytest.mark.skipif(shutil.which("g++") is None, reason="needs g++")
+@pytest.mark.parametrize("n,d", [(3, 128), (70000, 256), (5, 4096)])
+def test_unpermute_codes_index_math_on_cpu(tmp_path, n, d):
+    """unpermute_codes_kernel's loops over the host's launch grid (more rows than grid y
+    included) put every sweep-order code back at its original column: codes[:, perm] = cs."""
+    import numpy as np
+    exe = tmp_path / "unpermute_check"
+    r = subprocess.run(["g++", "-std=c++17", "-O2", "-Wall", "-Werror",
+                        "-I", os.path.join(ROOT, "post_weight_quantization_18_b200", "csrc"),
+                        os.path.join(ROOT, "tests", "c", "unpermute_check.cpp"), "-o", str(exe)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    rng = np.random.default_rng(n + d)
+    cs = rng.integers(0, 16, (n, d), dtype=np.uint8)
+    perm = rng.permutation(d).astype(np.int32)
+    (tmp_path / "cs.bin").write_bytes(cs.tobytes())
+    (tmp_path / "perm.bin").write_bytes(perm.tobytes())
+    r = subprocess.run([str(exe), str(n), str(d), str(tmp_path / "cs.bin"),
+                        str(tmp_path / "perm.bin"), str(tmp_path / "out.bin")],
+                       capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stderr
+    got = np.frombuffer((tmp_path / "out.bin").read_bytes(), np.uint8).reshape(n, d)
+    want = np.empty_like(cs)
+    want[:, perm] = cs
+    np.testing.assert_array_equal(got, want)
