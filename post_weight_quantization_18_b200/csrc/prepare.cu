@@ -130,11 +130,11 @@ __global__ void zero_lower_kernel(float* U, int d) {
 // U block = V^-1 where H_d = V V^T, V upper. A recursion on halves (the one the host uses above
 // 4096 columns), inside one CTA of 16 warps on two shared-memory matrices (A: the block being
 // factored, U: the result): 128 -> 64 -> 32 -> 16-column leaves. Each split does its four
-//   block products on the tensor cores (warp-level m16n8k8 TF32 with the three-term hi/lo split, so
-//   the products carry fp32 accuracy), skipping the k-ranges where the triangular operand is
-//   zero and computing only the upper tiles of the symmetric update. A 32-column node (two
-//   leaves and its four 16 x 16 products) runs on one warp without block barriers; a leaf is
-//   factored and inverted in registers.
+// block products on the tensor cores (warp-level m16n8k8 TF32 with the three-term hi/lo split,
+// so the products carry fp32 accuracy), skipping the k-ranges where the triangular operand is
+// zero and computing only the upper tiles of the symmetric update. A 32-column node (two
+// leaves and its four 16 x 16 products) runs on one warp without block barriers; a leaf is
+// factored and inverted in registers.
 // A block smaller than 128 is padded at its end with the identity: the padded factor is block
 // diagonal, so the leading n x n part is unchanged.
 constexpr int BASE_THREADS = 512;
