@@ -6,11 +6,7 @@
 #include <stdint.h>
 #include <string.h>
 
-#if defined(__CUDACC__)
-#define GPTQ_HD __host__ __device__ __forceinline__
-#else
-#define GPTQ_HD inline
-#endif
+#include "hd.cuh"
 
 namespace gptq {
 
@@ -31,7 +27,7 @@ GPTQ_HD float widen(uint16_t b) {
 // Source columns of k0 .. k0+3 and whether each is live (not dead).
 GPTQ_HD void gather4_cols(const int32_t* perm, const uint8_t* dead, int k0, int32_t (&src)[4],
                           bool (&live)[4]) {
-#pragma unroll
+GPTQ_UNROLL
   for (int j = 0; j < 4; ++j) {
     src[j] = perm[k0 + j];
     live[j] = dead[k0 + j] == 0;
@@ -42,7 +38,7 @@ template <typename T>  // float, or uint16_t holding bf16 bit patterns
 GPTQ_HD void gather4_row(const T* W, long long ldw, long long r, const int32_t (&src)[4],
                          const bool (&live)[4], float (&v)[4]) {
   const T* wr = W + r * ldw;
-#pragma unroll
+GPTQ_UNROLL
   for (int j = 0; j < 4; ++j) v[j] = live[j] ? widen(wr[src[j]]) : 0.0f;
 }
 

@@ -8,11 +8,7 @@
 
 #include <stdint.h>
 
-#if defined(__CUDACC__)
-#define GPTQ_HD __host__ __device__ __forceinline__
-#else
-#define GPTQ_HD inline
-#endif
+#include "hd.cuh"
 
 namespace gptq {
 
@@ -21,9 +17,9 @@ namespace gptq {
 template <int BITS>
 GPTQ_HD void pack32(const uint32_t (&c)[8], uint32_t (&w)[BITS]) {
   constexpr uint32_t mask = (1u << BITS) - 1u;
-#pragma unroll
+GPTQ_UNROLL
   for (int i = 0; i < BITS; ++i) w[i] = 0u;
-#pragma unroll
+GPTQ_UNROLL
   for (int k = 0; k < 32; ++k) {
     const uint32_t code = (c[k >> 2] >> (8 * (k & 3))) & mask;
     const int bit = k * BITS, wi = bit >> 5, off = bit & 31;

@@ -34,6 +34,7 @@ namespace {
 constexpr int BLK = 128;
 constexpr int ROWS_PER_WARP = 4;
 constexpr int LANES_PER_ROW = 8;
+static_assert(ROWS_PER_WARP * LANES_PER_ROW == 32, "eight lanes own one row");
 constexpr int SW_SMEM = BLK * BLK * 4 + BLK * 4 + 64;
 constexpr int SW_SMEM_STATIC = SW_SMEM + 3 * 16 * BLK * 4 + BLK * 4;  // + (s, 1/s, z) table
 

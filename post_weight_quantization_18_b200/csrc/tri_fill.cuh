@@ -5,11 +5,7 @@
 // the CPU.
 #pragma once
 
-#if defined(__CUDACC__)
-#define GPTQ_HD __host__ __device__ __forceinline__
-#else
-#define GPTQ_HD inline
-#endif
+#include "hd.cuh"
 
 namespace gptq {
 
