@@ -24,12 +24,19 @@ def as_f64(x) -> np.ndarray:
 
 
 def hessian(X_tm: np.ndarray, chunk: int = 16384) -> np.ndarray:
-    """H = 2 X^T X over token-major X (float64), summed over token chunks with a library matmul."""
+    """H = 2 X^T X over token-major X (float64), summed over token chunks.
+
+    H is symmetric, so each chunk adds only its upper triangle, with the BLAS symmetric rank-k
+    update (dsyrk) as the library step; the lower triangle is the mirror of the upper one."""
+    from scipy.linalg import blas
     N, d = X_tm.shape
-    H = np.zeros((d, d), np.float64)
+    H = np.zeros((d, d), np.float64, order="F")
     for t0 in range(0, N, chunk):
-        xc = as_f64(X_tm[t0:t0 + chunk])
-        H += xc.T @ xc
+        xc = np.ascontiguousarray(as_f64(X_tm[t0:t0 + chunk]))
+        # xc is [t, d] row-major, i.e. the column-major [d, t] matrix A = xc^T; C += A A^T.
+        H = blas.dsyrk(1.0, xc.T, beta=1.0, c=H, trans=0, lower=0, overwrite_c=1)
+    H = np.triu(H)
+    H += np.triu(H, 1).T
     return 2.0 * H
 
 

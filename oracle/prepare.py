@@ -46,21 +46,40 @@ def dead_fix(H: np.ndarray, W: np.ndarray):
 def damp(H: np.ndarray, percdamp: float):
     """H + lambda I with lambda = percdamp * mean(diag(H)). Returns (H_damped, lambda)."""
     lam = percdamp * float(np.mean(np.diag(H)))
-    return H + lam * np.eye(H.shape[0]), lam
+    Hd = np.array(H, np.float64, copy=True)
+    idx = np.arange(Hd.shape[0])
+    Hd[idx, idx] += lam
+    return Hd, lam
+
+
+def chol_lower(A: np.ndarray) -> np.ndarray:
+    """Lower Cholesky factor L of a symmetric positive definite A (A = L L^T), by LAPACK's
+    dpotrf. A is symmetric, so its row-major array read column-major is A itself."""
+    from scipy.linalg import lapack
+    c, info = lapack.dpotrf(np.asarray(A, np.float64).T, lower=1, clean=1, overwrite_a=0)
+    if info != 0:
+        raise np.linalg.LinAlgError(f"dpotrf: leading minor {info} is not positive definite")
+    return np.ascontiguousarray(c)
 
 
 def cholesky_inverse(L: np.ndarray) -> np.ndarray:
-    """(L L^T)^-1 from the lower Cholesky factor L: L^-T L^-1."""
-    Linv = scipy.linalg.solve_triangular(L, np.eye(L.shape[0]), lower=True)
-    return Linv.T @ Linv
+    """(L L^T)^-1 = L^-T L^-1 from the lower Cholesky factor L, by LAPACK's dpotri (the
+    'cholesky_inverse' step of the walkthrough); the full symmetric matrix is returned."""
+    from scipy.linalg import lapack
+    inv, info = lapack.dpotri(np.asfortranarray(L), lower=1, overwrite_c=0)
+    if info != 0:
+        raise np.linalg.LinAlgError(f"dpotri: info {info}")
+    inv = np.tril(inv)
+    inv += np.tril(inv, -1).T
+    return np.ascontiguousarray(inv)
 
 
 def upper_chol_of_inverse(H_damped: np.ndarray):
     """The walkthrough's three steps. Returns (H_inv, U) with H_inv = U^T U, U upper."""
-    L = np.linalg.cholesky(H_damped)
+    L = chol_lower(H_damped)
     H_inv = cholesky_inverse(L)
-    H_inv = 0.5 * (H_inv + H_inv.T)
-    U = np.linalg.cholesky(H_inv).T
+    del L
+    U = np.ascontiguousarray(chol_lower(H_inv).T)
     return H_inv, U
 
 
@@ -77,8 +96,9 @@ def prepare(H: np.ndarray, W: np.ndarray, percdamp: float = 0.01, act_order: boo
     if perm is None:
         perm = act_order_perm(np.diag(H)) if act_order else np.arange(d, dtype=np.int64)
     perm = np.asarray(perm, np.int64)
-    Hp = H[np.ix_(perm, perm)]
-    Wp = W[:, perm]
+    identity = np.array_equal(perm, np.arange(d))
+    Hp = H if identity else H[np.ix_(perm, perm)]
+    Wp = W if identity else W[:, perm]
     Hp, Wp, dead = dead_fix(Hp, Wp)
     Hd, lam = damp(Hp, percdamp)
     H_inv, U = upper_chol_of_inverse(Hd)
