@@ -18,6 +18,13 @@ act-order): the groups are runs of g columns in the original column order, their
 taken once from the original (dead-column-fixed) weights before the sweep, and a column swept at
 position j uses the parameters of its original group. The routes take them as `static`.
 
+Precision: the compensation runs in float64; the integer decisions (the group's zero point and
+every code) and the group scale are taken in float32, from the float64 compensated weights
+rounded once to float32, with IEEE division and round-half-to-even: the pages' quantizer is
+float32 tensor code, and a decision that floating point takes must be taken in the same
+precision as the kernel under test takes it (the RTN and quantize-given-scales paths of
+quantizer.py already run in float32).
+
 Routes
   sweep_obs       OBS update with the explicit inverse Hessian H_F^-1, downdated after every
                   column by the rank-1 formula of [GPTQ-MATH] §Recursive Inverse Hessian
@@ -44,6 +51,12 @@ import numpy as np
 from . import quantizer as qz
 
 
+def _decide_params(vals: np.ndarray, bits: int, sym: bool):
+    """(s, z) of each row of vals, decided in float32 (see the module docstring)."""
+    s, z = qz.params_from_values(np.asarray(vals, np.float64).astype(np.float32), bits, sym)
+    return s.astype(np.float64), z.astype(np.float64)
+
+
 def static_group_params(W_orig: np.ndarray, bits: int, group_size: int, sym: bool):
     """(S, Z) [n, G] of the runs of group_size columns of W in its original column order."""
     n, d = W_orig.shape
@@ -51,8 +64,8 @@ def static_group_params(W_orig: np.ndarray, bits: int, group_size: int, sym: boo
     S = np.zeros((n, G))
     Z = np.zeros((n, G))
     for gi in range(G):
-        S[:, gi], Z[:, gi] = qz.params_from_values(
-            np.asarray(W_orig[:, gi * group_size:(gi + 1) * group_size], np.float64), bits, sym)
+        S[:, gi], Z[:, gi] = _decide_params(W_orig[:, gi * group_size:(gi + 1) * group_size],
+                                            bits, sym)
     return S, Z
 
 
@@ -76,7 +89,7 @@ class _Groups:
         self.S = np.zeros((n, G))
         self.Z = np.zeros((n, G))
         if self.per_row:
-            s, z = qz.params_from_values(W0, bits, sym)
+            s, z = _decide_params(W0, bits, sym)
             self.S[:, 0], self.Z[:, 0] = s, z
 
     def at(self, W: np.ndarray, j: int):
@@ -87,14 +100,17 @@ class _Groups:
             return self.S[:, 0], self.Z[:, 0]
         gi = j // self.g
         if j % self.g == 0:
-            s, z = qz.params_from_values(W[:, j:j + self.g], self.bits, self.sym)
+            s, z = _decide_params(W[:, j:j + self.g], self.bits, self.sym)
             self.S[:, gi], self.Z[:, gi] = s, z
         return self.S[:, gi], self.Z[:, gi]
 
 
 def _quant_col(W, j, grp):
+    """Code of column j decided in float32 from the float64 compensated weights; w_hat in
+    float64 (exact: s is a float32 value and q - z a small integer)."""
     s, z = grp.at(W, j)
-    q = qz.quantize(W[:, j], s, z, grp.bits)
+    q = qz.quantize(W[:, j].astype(np.float32), s.astype(np.float32), z.astype(np.float32),
+                    grp.bits).astype(np.float64)
     return q, qz.dequantize(q, s, z)
 
 

@@ -50,12 +50,13 @@ def test_routes_agree(bits, gs, sym, half):
 def test_identity_hessian_reduces_to_rtn():
     """H = I: U is diagonal, no compensation happens, GPTQ codes are RTN codes."""
     rng = np.random.default_rng(1)
-    W = rng.normal(0, 0.02, (16, 256))
+    W = rng.normal(0, 0.02, (16, 256)).astype(np.float32)   # weights are fp32 or bf16 values
     for bits, gs, sym in [(4, 128, False), (3, 64, False), (4, -1, True)]:
-        L = oracle.gptq_layer(W, np.eye(256), bits, gs, sym)
+        L = oracle.gptq_layer(W.astype(np.float64), np.eye(256), bits, gs, sym)
         R = oracle.rtn_layer(W, bits, gs, sym)
         np.testing.assert_array_equal(L["codes"], R["codes"])
-        np.testing.assert_allclose(L["S"], R["S"], rtol=1e-15)
+        np.testing.assert_array_equal(L["S"], R["S"])
+        np.testing.assert_array_equal(L["Z"], R["Z"])
 
 
 def test_single_column_saliency():
@@ -66,8 +67,8 @@ def test_single_column_saliency():
     H_inv = np.linalg.inv(H)
     c, S, Z, W1 = sw.sweep_obs(W, H_inv, 4, 12, False, n_steps=1)
     delta = W1 - W
-    s, z = qz.params_from_values(W, 4, False)
-    wq = qz.dequantize(qz.quantize(W[:, 0], s, z, 4), s, z)
+    wq = qz.dequantize(c[:, 0].astype(np.float64), S[:, 0], Z[:, 0])   # the step's own w_hat
+    assert np.all(np.abs(W[:, 0] - wq) <= S[:, 0] / 2 * (1 + 1e-6))   # a rounding of w_q
     expected = (W[:, 0] - wq) ** 2 / (2 * H_inv[0, 0])
     measured = np.sum((X @ delta.T) ** 2, axis=0)
     np.testing.assert_allclose(measured, expected, rtol=1e-9)
@@ -167,11 +168,12 @@ def test_static_groups_identity_hessian_is_rtn_in_any_order():
     """H = I with static groups: no compensation and the groups' parameters are RTN's, so the
     codes equal RTN of the original weights whatever the column order."""
     rng = np.random.default_rng(4)
-    W = rng.normal(0, 0.02, (12, 96))
+    W = rng.normal(0, 0.02, (12, 96)).astype(np.float32)
     R = qz.rtn(W, 4, 32, False)
     for seed in range(3):
         perm = np.random.default_rng(seed).permutation(96)
-        L = oracle.gptq_layer(W, np.eye(96), 4, 32, False, perm=perm, static_groups=True)
+        L = oracle.gptq_layer(W.astype(np.float64), np.eye(96), 4, 32, False, perm=perm,
+                              static_groups=True)
         np.testing.assert_array_equal(L["codes"], R[0])
         np.testing.assert_array_equal(L["S"], R[1])
         np.testing.assert_array_equal(L["g_idx"], np.arange(96) // 32)
