@@ -4,18 +4,21 @@
 A step is the whole hot path for one layer: H = 2 X^T X over all calibration tokens
 (gptq_hessian_accumulate), damping + U = upper Cholesky factor of H^-1 (gptq_prepare_hinv), the
 column sweep with lazy updates (gptq_quantize_layer) and packing (gptq_pack), all through the C
-ABI. Default workload: Llama-7B attention projection, W 4096 x 4096 bf16, X 262144 x 4096 bf16
-(128 sequences x 2048 tokens, lognormal(0, 1) channel scales, 0.1 % outlier channels x20),
-4-bit asymmetric, group 128, block 128, damp 0.01.
+ABI. Default workload: the largest single-GPU layer, a Llama-70B-shaped down projection,
+W 8192 x 28672 bf16 ~ N(0, 0.015^2), X 131072 x 28672 bf16 half-normal with lognormal(0, 1)
+channel scales and 0.05 % outlier channels x30, 4-bit symmetric with one scale per row,
+block 128, damp 0.01 (a 28672^2 fp32 Hessian). --workload selects another one.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 Prints one JSON line (rank 0). Under torchrun each rank quantizes its own layer (independent
 problems, no collective on the data path: weak scaling); the timed duration is the max over ranks.
 --impl reference times the FP64 CPU oracle on bounded samples of the same workload.
-Outside the timed steps the line also reports the per-stage times (breakdown_ms), the SYRK
-roofline, the end-to-end rate from pinned host buffers (e2e), the oracle's rate (cpu_baseline),
-and the dequantizing GEMV on a packed 8192 x 28672 int4 layer (dequant_gemv).
+Besides the headline the line reports the per-stage times (breakdown_ms) and each stage's
+roofline (stages), the SYRK kernel's roofline (roofline), the end-to-end rate through the C ABI
+from pinned host buffers (e2e), the oracle's rate on the host cores (cpu_baseline), the number
+of kernels launched in the timed steps (counted from the recorded CUDA graphs), and the
+dequantizing GEMV on a packed 8192 x 28672 int4 layer (dequant_gemv).
 """
 from __future__ import annotations
 
@@ -34,7 +37,9 @@ sys.path.insert(0, ROOT)
 
 METRIC = "GPTQ layer quantize wall ms & weights/s (incl. XXᵀ); SYRK TFLOP/s; sweep GB/s"
 UNIT = "weights/s"
-DEFAULT_WORKLOAD = "llama7b_attn_proj"
+DEFAULT_WORKLOAD = "llama70b_down_proj"
+# TF32 peak from the measured bf16 peak by the nominal dense ratio (1.1 / 2.25 PFLOP/s).
+TF32_PER_BF16 = 1.1 / 2.25
 
 
 def parse_args():
@@ -44,7 +49,7 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
-    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-steps", type=int, default=5, help="end-to-end steps (at least 1)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="calibration tokens instead of the workload's own count (smaller cases "
                          "for profiler captures; the config line reports the count used)")
@@ -55,77 +60,48 @@ def parse_args():
     return ap.parse_args()
 
 
-def syrk_traffic():
-    """DRAM bytes per launch of the SYRK kernel from its committed ncu summary, or None when the
-    kernel source has changed since the counters were taken (the summary records its hash)."""
-    import hashlib
-    import re
-    try:
-        with open(os.path.join(ROOT, "profiles", "syrk_bf16_llama7b_attn_proj.md")) as f:
-            text = f.read()
-        with open(os.path.join(ROOT, "post_weight_quantization_18_b200", "csrc",
-                               "syrk_bf16.cu"), "rb") as f:
-            digest = hashlib.sha256(f.read()).hexdigest()
-    except OSError:
-        return None
-    want = re.search(r"kernel_source_sha256:\s*([0-9a-f]{64})", text)
-    val = re.search(r"traffic_bytes_per_launch:\s*([0-9]+)", text)
-    if not want or not val or want.group(1) != digest:
-        return None
-    return int(val.group(1))
-
-
 def peaks():
+    """(HBM GB/s, bf16 TFLOP/s burst, bf16 TFLOP/s sustained, source)."""
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             p = json.load(f)
-        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+        return (float(p["hbm_gbs"]), float(p["bf16_tflops"]),
+                float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), "measured")
     except Exception:
-        return 6650.0, 1590.0, "fallback"
+        return 6650.0, 1590.0, 1400.0, "fallback"
 
 
 # ------------------------------------------------------------------------------------------
-# Launch accounting (mirrors the host recursions in csrc/api.cu)
+# Kernel launches of a step, counted from the CUDA graphs recorded from its C ABI calls
 # ------------------------------------------------------------------------------------------
 
-def _split(n):
-    m = ((n // 2) + 127) // 128 * 128
-    if m >= n:
-        m = n - 128
-    if m <= 0:
-        m = n // 2
-    return m
+def new_graph():
+    import torch
+    try:
+        return torch.cuda.CUDAGraph(keep_graph=True), True
+    except TypeError:
+        return torch.cuda.CUDAGraph(), False
 
 
-def _rl_launches(n):
-    """Right-looking node of nb blocks: per block a base block; below the last, the panel block
-    and the diagonal update; below the last two, the rest of the panel and the trailing update
-    (with the next block column); and two products of the inverse for every block but the
-    last."""
-    nb = (n + 127) // 128
-    return nb + 2 * (nb - 1) + 2 * max(0, nb - 2) + 2 * (nb - 1)
-
-
-def _prep_launches(n):
-    if n <= 32 * 128:
-        return _rl_launches(n)
-    m = _split(n)
-    return 4 + _prep_launches(m) + _prep_launches(n - m)
-
-
-def _sweep_launches(n):
-    if n <= 128:
-        return 1
-    m = _split(n)
-    return 1 + _sweep_launches(m) + _sweep_launches(n - m)
-
-
-def launches_per_step(d, q):
-    hess = 2
-    prep = (1 if not q.act_order else 3) + 2 + _prep_launches(d)
-    quant = 1 + (1 if q.group_size == -1 else 0) + _sweep_launches(d) + \
-        (1 if q.act_order else 0) + 1
-    return hess + prep + quant + 2
+def graph_kernel_nodes(gr):
+    """Number of kernel nodes in a recorded graph (None when the graph is not inspectable)."""
+    try:
+        from cuda.bindings import runtime as rt
+        handle = gr.raw_cuda_graph()
+        err, _, n = rt.cudaGraphGetNodes(handle, 0)
+        if int(err) != 0:
+            return None
+        err, nodes, n = rt.cudaGraphGetNodes(handle, n)
+        if int(err) != 0:
+            return None
+        kern = 0
+        for nd in nodes:
+            err, t = rt.cudaGraphNodeGetType(nd)
+            if int(err) == 0 and t == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel:
+                kern += 1
+        return kern
+    except Exception:
+        return None
 
 
 # ------------------------------------------------------------------------------------------
@@ -197,35 +173,78 @@ class ClockSampler:
 # Oracle timing (CPU baseline and the reference arm)
 # ------------------------------------------------------------------------------------------
 
-def oracle_sample(wl, X_host, W_host, tok_sample, row_sample):
-    """Time the FP64 oracle on a bounded sample of one layer and extrapolate to the whole layer.
-    Returns (seconds for the full layer, description)."""
-    import numpy as np
+class OracleSample:
+    """The FP64 oracle on a bounded sample of one layer of the workload. Both the cpu_baseline
+    key of our arm and the reference arm use this one definition:
+      * H over the first `tokens` calibration tokens (all d channels), scaled by N / tokens
+        (H is a sum over tokens);
+      * the prepare (act-order, dead columns, damping, U) at the full d, on that sample's H:
+        timed once per process and reused by every step (its cost does not depend on the
+        values);
+      * the blocked sweep and the pack of the first `rows` rows of W at the full d, scaled by
+        d_out / rows.
+    A step is one H sample plus one sweep-and-pack sample; the whole layer's time is
+    extrapolated from the step and the one prepare."""
 
-    import oracle
-    from oracle import hessian as hs
-    from oracle import prepare as prep
-    from oracle import sweep as sw
-    q = wl.quant
-    N, d = X_host.shape
-    n = W_host.shape[0]
-    tok = min(N, tok_sample)
-    rows = min(n, row_sample)
-    Xs = X_host[:tok].double().numpy()
-    t0 = time.perf_counter()
-    H = hs.hessian(Xs)
-    t_h = time.perf_counter() - t0
-    W64 = W_host[:rows].double().numpy()
-    t0 = time.perf_counter()
-    P = prep.prepare(H, W64, q.percdamp, act_order=q.act_order)
-    t_p = time.perf_counter() - t0
-    t0 = time.perf_counter()
-    sw.sweep_blocked(P["W"], P["U"], q.bits, q.group_size, q.sym, q.block_size)
-    t_s = time.perf_counter() - t0
-    total = t_h * (N / tok) + t_p + t_s * (n / rows)
-    desc = (f"oracle on {tok} of {N} tokens (H, scaled x{N / tok:.0f}), full {d}x{d} prepare, "
-            f"sweep of {rows} of {n} rows (scaled x{n / rows:.0f})")
-    return total, desc, dict(hessian_s=t_h, prepare_s=t_p, sweep_s=t_s)
+    def __init__(self, wl, tokens, rows):
+        import torch
+
+        import layer_inputs as li
+        self.wl = wl
+        lin = wl.linears[0]
+        act = wl.act(lin.act)
+        self.N, self.d, self.n = act.n_tokens, lin.d_in, lin.d_out
+        self.tokens, self.rows = min(tokens, act.n_tokens), min(rows, lin.d_out)
+        # The first rows of the full workload's X and W (same seeded streams, same order).
+        self.X = li.activations(self.tokens, act.d, chan_sigma=act.chan_sigma,
+                                outlier_frac=act.outlier_frac, outlier_mult=act.outlier_mult,
+                                half_normal=act.half_normal, dtype=torch.bfloat16, seed=act.seed)
+        self.W = li.weight(self.rows, lin.d_in, lin.sigma, torch.bfloat16, lin.seed)
+        self.P = None
+        self.prepare_s = None
+
+    def _hessian(self):
+        from oracle import hessian as hs
+        t0 = time.perf_counter()
+        H = hs.hessian(self.X)
+        return H, time.perf_counter() - t0
+
+    def prepare_once(self):
+        from oracle import prepare as prep
+        q = self.wl.quant
+        H, _ = self._hessian()
+        t0 = time.perf_counter()
+        self.P = prep.prepare(H, self.W.double().numpy(), q.percdamp, act_order=q.act_order)
+        self.prepare_s = time.perf_counter() - t0
+        self.P.pop("H_inv", None)
+        self.P.pop("H_damped", None)
+
+    def step(self):
+        """One sample step. Returns (seconds the step took, its parts)."""
+        from oracle import pack as pk
+        from oracle import sweep as sw
+        q = self.wl.quant
+        t0 = time.perf_counter()
+        _, t_h = self._hessian()
+        t1 = time.perf_counter()
+        codes, S, Z, _ = sw.sweep_blocked(self.P["W"], self.P["U"], q.bits, q.group_size, q.sym,
+                                          q.block_size)
+        pk.pack(codes, S, Z, q.bits)
+        t2 = time.perf_counter()
+        return t2 - t0, dict(hessian_s=t_h, sweep_pack_s=t2 - t1)
+
+    def layer_seconds(self, parts):
+        return (parts["hessian_s"] * self.N / self.tokens + self.prepare_s +
+                parts["sweep_pack_s"] * self.n / self.rows)
+
+    def describe(self):
+        return (f"FP64 oracle: H over {self.tokens} of {self.N} tokens (x{self.N / self.tokens:.0f}),"
+                f" the full {self.d}x{self.d} prepare once per process "
+                f"({self.prepare_s:.1f} s), blocked sweep and pack of {self.rows} of {self.n} rows "
+                f"(x{self.n / self.rows:.0f}); layer time extrapolated from these")
+
+
+ORACLE_TOKENS, ORACLE_ROWS = 4096, 256
 
 
 def cpu_cores():
@@ -240,49 +259,34 @@ def cpu_cores():
 
 
 def run_reference(args):
-    import torch
-
-    import layer_inputs as li
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     wl = workload(args)
     lin = wl.linears[0]
-    act = wl.act(lin.act)
-    tok_sample, row_sample = 4096, 32
-    X = li.activations(tok_sample, act.d, chan_sigma=act.chan_sigma,
-                       outlier_frac=act.outlier_frac, outlier_mult=act.outlier_mult,
-                       half_normal=act.half_normal, dtype=torch.bfloat16, seed=act.seed)
-    W = li.weight(row_sample, lin.d_in, lin.sigma, torch.bfloat16, lin.seed)
-
-    class Full:  # shapes of the full workload for extrapolation
-        shape = (act.n_tokens, act.d)
-
-    def step():
-        secs, desc, parts = oracle_sample(wl, X, W, tok_sample, row_sample)
-        # scale from the generated sample shape to the full workload
-        secs = parts["hessian_s"] * (act.n_tokens / tok_sample) + parts["prepare_s"] + \
-            parts["sweep_s"] * (lin.d_out / row_sample)
-        return secs, parts
+    smp = OracleSample(wl, ORACLE_TOKENS, ORACLE_ROWS)
+    smp.prepare_once()
     for _ in range(args.warmup):
-        step()
-    times = []
+        smp.step()
+    step_s, layer_s = [], []
     for _ in range(args.steps):
-        secs, parts = step()
-        times.append(secs)
-    per = statistics.mean(times)
-    value = lin.d_out * lin.d_in / per
-    sample = (f"each step: FP64 oracle H on {tok_sample} of {act.n_tokens} tokens (scaled), full "
-              f"{act.d}x{act.d} prepare, blocked sweep of {row_sample} of {lin.d_out} rows (scaled)")
-    # Same line as this bench's own arm (n_gpus and config of the launch); what actually ran,
-    # the oracle on this host's cores, is described under cpu_baseline.
+        secs, parts = smp.step()
+        step_s.append(secs)
+        layer_s.append(smp.layer_seconds(parts))
+    per_layer = statistics.mean(layer_s)
+    value = lin.d_out * lin.d_in / per_layer
+    # Same line as this bench's own arm (n_gpus and config of the launch); ms_per_step is the
+    # time of a sample step as it ran, value the whole-layer rate extrapolated from it.
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": per * 1e3, "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": statistics.mean(step_s) * 1e3,
+            "extrapolated_layer_ms": per_layer * 1e3,
+            "oracle_prepare_ms_once": smp.prepare_s * 1e3,
+            "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_dict(args, wl, world=args.gpus),
             "cpu_baseline": {"kind": "oracle", "value": value, "unit": UNIT, "cores": cpu_cores(),
-                             "sample": sample},
+                             "sample": smp.describe()},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -297,6 +301,53 @@ def workload(args):
         acts = tuple(dataclasses.replace(a, n_tokens=args.tokens) for a in wl.acts)
         wl = dataclasses.replace(wl, acts=acts)
     return wl
+
+
+def measure_gemm(L, dev, n, d, reps=5):
+    """The product kernel (gemm_tf32x3_kernel through gptq_gemm_f32) at the shape of the step's
+    largest lazy update, W[:, m:] -= Err[:, :m] U[:m, m:] with m = d / 2: M = n, N = K = d / 2.
+    Random fp32 operands; CUDA events around each launch on the current stream."""
+    import torch
+    m = d // 2
+    A = torch.randn((n, m), device=dev) * 1e-3
+    B = torch.randn((m, m), device=dev)
+    C = torch.randn((n, m), device=dev)
+    for _ in range(2):
+        L.gptq_gemm_f32(A, B, C, alpha=-1.0, beta=1.0)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+    torch.cuda.synchronize()
+    ev[0].record()
+    for i in range(reps):
+        L.gptq_gemm_f32(A, B, C, alpha=-1.0, beta=1.0)
+        ev[i + 1].record()
+    torch.cuda.synchronize()
+    ms = statistics.mean(ev[i].elapsed_time(ev[i + 1]) for i in range(reps))
+    flops = 2.0 * n * m * m
+    del A, B, C
+    return {"M": n, "N": m, "K": m, "ms": ms, "flops": flops, "tflops": flops / (ms * 1e-3) / 1e12,
+            "reps": reps}
+
+
+def measure_pack(L, dev, Wd, U, perm, dead, p, codes, scales, zeros, g_idx, ws, status, qweight,
+                 s16, z16, bits, reps=20):
+    """gptq_pack alone on this layer's codes (one gptq_quantize_layer run outside the timing);
+    CUDA events around each launch on the current stream. HBM-bound."""
+    import torch
+    L.gptq_quantize_layer(Wd, U, perm, dead, p, codes, scales, zeros, g_idx, ws, status)
+    for _ in range(3):
+        L.gptq_pack(codes, bits, scales, zeros, qweight, s16, z16)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+    torch.cuda.synchronize()
+    ev[0].record()
+    for i in range(reps):
+        L.gptq_pack(codes, bits, scales, zeros, qweight, s16, z16)
+        ev[i + 1].record()
+    torch.cuda.synchronize()
+    us = statistics.mean(ev[i].elapsed_time(ev[i + 1]) for i in range(reps)) * 1e3
+    n, d = codes.shape
+    G = scales.shape[1]
+    nbytes = n * d + n * ((d * bits + 31) // 32) * 4 + n * G * 12
+    return {"us": us, "bytes": nbytes}
 
 
 def measure_gemv(L, dev, hbm_gbs):
@@ -426,17 +477,17 @@ def run_ours(args):
     flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device=dev)  # 256 MiB > L2
     outs_h = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (qweight, s16, z16, g_idx)]
 
-    ev = {k: [] for k in ("step", "syrk", "prep", "quant", "pack")}
+    ev = {k: [] for k in ("step", "syrk", "prep", "quant")}
+    # The step: H, prepare, and the sweep writing the packed layer (codes are never stored).
     calls = [
         lambda X, W: L.gptq_hessian_accumulate(H, X, 2.0, False, status),
         lambda X, W: L.gptq_prepare_hinv(H, p, U, perm, dead, ws, status),
-        lambda X, W: L.gptq_quantize_layer(W, U, perm, dead, p, codes, scales, zeros, g_idx, ws,
-                                           status),
-        lambda X, W: L.gptq_pack(codes, q.bits, scales, zeros, qweight, s16, z16),
+        lambda X, W: L.gptq_quantize_pack_layer(W, U, perm, dead, p, qweight, s16, z16, scales,
+                                                zeros, g_idx, ws, status),
     ]
 
     def step(X, W, record, graphs=None):
-        e = [torch.cuda.Event(enable_timing=True) for _ in range(5)] if record else None
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)] if record else None
         if record:
             e[0].record()
         for i, call in enumerate(calls):
@@ -447,11 +498,10 @@ def run_ours(args):
             if record:
                 e[i + 1].record()
         if record:
-            ev["step"].append((e[0], e[4]))
+            ev["step"].append((e[0], e[3]))
             ev["syrk"].append((e[0], e[1]))
             ev["prep"].append((e[1], e[2]))
             ev["quant"].append((e[2], e[3]))
-            ev["pack"].append((e[3], e[4]))
 
     for _ in range(max(3, args.warmup)):
         step(Xd, Wd, False)
@@ -463,17 +513,23 @@ def run_ours(args):
     # Record each C ABI call of the step once into a CUDA graph (the calls only enqueue
     # kernels on the current stream) and replay the graphs in the timed steps: the ~230
     # launches of a step then cost no host time and no launch gaps.
-    graphs = None
-    if not args.eager:
-        graphs = []
-        for call in calls:
-            gr = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(gr):
-                call(Xd, Wd)
-            graphs.append(gr)
-        for gr in graphs:      # one untimed replay of the recorded step
-            gr.replay()
-        torch.cuda.synchronize()
+    # The same recording gives the number of kernels a step launches (kernel nodes).
+    graphs = []
+    launches = 0
+    for call in calls:
+        gr, kept = new_graph()
+        with torch.cuda.graph(gr):
+            call(Xd, Wd)
+        k = graph_kernel_nodes(gr) if kept else None
+        launches = None if (launches is None or k is None) else launches + k
+        if kept and hasattr(gr, "instantiate"):
+            gr.instantiate()
+        graphs.append(gr)
+    for gr in graphs:      # one untimed replay of the recorded step
+        gr.replay()
+    torch.cuda.synchronize()
+    if args.eager:
+        graphs = None
 
     with ClockSampler(local) as clk:
         if world > 1:
@@ -510,45 +566,96 @@ def run_ours(args):
     e2e_total_s = sum(e2e_ms) / 1e3
     total_s, e2e_total_s = max_over_ranks([total_s, e2e_total_s], dev)
 
-    hbm, bf16, peak_kind = peaks()
+    hbm, bf16, bf16_sus, peak_kind = peaks()
+    tf32x3 = bf16 * TF32_PER_BF16 / 3.0   # fp32-accurate products: three TF32 MMAs each
+    # Side measurements, after the timed steps (same stream, CUDA events):
+    gemm = measure_gemm(L, dev, n, d)     # the dominant kernel at the step's largest product
+    pack = measure_pack(L, dev, Wd, U, perm, dead, p, codes, scales, zeros, g_idx, ws, status,
+                        qweight, s16, z16, q.bits)
     gemv = measure_gemv(L, dev, hbm)
     if rank == 0:
-        syrk_ms = statistics.mean(ms("syrk"))
-        quant_ms = statistics.mean(ms("quant"))
+        stage_ms = {k: statistics.mean(ms(k)) for k in ("syrk", "prep", "quant")}
         syrk_flops = float(d) * (d + 1) * N
-        syrk_tflops = syrk_flops / (syrk_ms * 1e-3) / 1e12
-        sweep_bytes = n * d * 9 + n * G_n * 8 + d * d * 4
+        syrk_tflops = syrk_flops / (stage_ms["syrk"] * 1e-3) / 1e12
+        # Sweep with packed output: W read, Err written and the packed bits written per weight;
+        # fp32 and fp16 s, z per (row, group); the U diagonal blocks once. Its lazy updates are
+        # n d^2 flops of 3xTF32 products.
+        sweep_bytes = (n * d * 8 + n * ((d * q.bits + 31) // 32) * 4 + n * G_n * 12 +
+                       (d // 128) * 128 * 128 * 4)
+        sweep_flops = float(n) * d * d
+        prep_flops = 2.0 / 3.0 * float(d) ** 3
         weights = n * d
         value = world * args.steps * weights / total_s
         e2e_value = world * args.e2e_steps * weights / e2e_total_s
         h2d = Xh.numel() * Xh.element_size() + Wh.numel() * Wh.element_size()
         d2h = sum(o.numel() * o.element_size() for o in outs_h)
+
+        def stage(ms_, bound, work, unit, peak, peak_src, algo, **extra):
+            t_roof = work / (peak * (1e12 if unit == "TFLOP/s" else 1e9))
+            ach = work / (ms_ * 1e-3) / (1e12 if unit == "TFLOP/s" else 1e9)
+            return dict(ms=ms_, bound=bound, achieved=ach, peak=peak, unit=unit,
+                        frac=ach / peak, roof_ms=t_roof * 1e3, peak_source=peak_src,
+                        algorithmic=algo, **extra)
+        sweep_t = max(sweep_flops / (tf32x3 * 1e12), sweep_bytes / (hbm * 1e9))
+        tf_src = f"{peak_kind} bf16 burst x 1.1/2.25 (TF32) / 3 (3xTF32)"
+        stages = {
+            "hessian_syrk": stage(stage_ms["syrk"], "tensor", syrk_flops, "TFLOP/s", bf16,
+                                  f"{peak_kind} bf16 burst", f"d(d+1)N = {syrk_flops:.4g} flop"),
+            "prepare": stage(stage_ms["prep"], "tensor", prep_flops, "TFLOP/s", tf32x3, tf_src,
+                             f"2/3 d^3 = {prep_flops:.4g} flop (Cholesky and inverse)"),
+            "quantize_sweep_pack": stage(stage_ms["quant"], "tensor", sweep_flops, "TFLOP/s",
+                                         tf32x3, tf_src,
+                                         f"n d^2 = {sweep_flops:.4g} flop of lazy updates",
+                                         bytes=sweep_bytes,
+                                         hbm_frac=sweep_bytes / (stage_ms["quant"] * 1e-3) /
+                                         (hbm * 1e9),
+                                         roof_ms_max_of_flops_and_bytes=sweep_t * 1e3),
+            "pack_standalone": stage(pack["us"] * 1e-3, "hbm", pack["bytes"], "GB/s", hbm,
+                                     f"{peak_kind} HBM copy",
+                                     f"{pack['bytes']} B (codes read, words and fp16 s/z "
+                                     "written, fp32 s/z read)",
+                                     note="gptq_pack on this layer's codes, timed alone; the "
+                                          "step packs inside the sweep instead"),
+        }
         cpu = None
         if not args.no_cpu_baseline and world == 1:
-            secs, desc, _ = oracle_sample(wl, Xh, Wh, 8192, 64)
-            cpu = {"value": weights / secs, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
-                   "sample": desc}
+            smp = OracleSample(wl, ORACLE_TOKENS, ORACLE_ROWS)
+            smp.prepare_once()
+            _, parts = smp.step()
+            cpu = {"value": weights / smp.layer_seconds(parts), "unit": UNIT,
+                   "cores": cpu_cores(), "kind": "oracle", "sample": smp.describe()}
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": max(3, args.warmup), "ms_per_step": statistics.mean(step_ms),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic (seeded W ~ N(0, 0.02^2), X lognormal channel scales with outliers)",
+            "data": f"synthetic (seeded W ~ N(0, {lin.sigma}^2), X lognormal channel scales with "
+                    "outliers)",
             "config": config_dict(args, wl, world),
-            "breakdown_ms": {"hessian_syrk": syrk_ms, "prepare": statistics.mean(ms("prep")),
-                             "quantize_sweep": quant_ms, "pack": statistics.mean(ms("pack"))},
+            "breakdown_ms": {"hessian_syrk": stage_ms["syrk"], "prepare": stage_ms["prep"],
+                             "quantize_sweep_pack": stage_ms["quant"]},
             "syrk_tflops": syrk_tflops,
             # the same time counted as the full 2 d^2 N product (upper and lower triangle)
-            "syrk_tflops_2d2n_equivalent": 2.0 * d * d * N / (syrk_ms * 1e-3) / 1e12,
-            "sweep_gbs": sweep_bytes / (quant_ms * 1e-3) / 1e9,
-            "roofline": {"bound": "tensor", "kernel": "syrk_bf16_tcgen05_kernel",
-                         "achieved": syrk_tflops, "peak": bf16, "unit": "TFLOP/s",
-                         "frac": syrk_tflops / bf16,
-                         "traffic": syrk_traffic() if act.n_tokens == 262144 and d == 4096 else None,
-                         "peak_source": f"{peak_kind} bf16 burst",
-                         "algorithmic": f"d(d+1)N = {syrk_flops:.4g} flop per launch"},
+            "syrk_tflops_2d2n_equivalent": 2.0 * d * d * N / (stage_ms["syrk"] * 1e-3) / 1e12,
+            "sweep_gbs": sweep_bytes / (stage_ms["quant"] * 1e-3) / 1e9,
+            "roofline": {"bound": "tensor", "kernel": "gemm_tf32x3_kernel",
+                         "achieved": gemm["tflops"], "peak": tf32x3, "unit": "TFLOP/s",
+                         "frac": gemm["tflops"] / tf32x3, "traffic": None,
+                         "peak_source": tf_src,
+                         "algorithmic": f"2 M N K = {gemm['flops']:.4g} flop per launch "
+                                        f"(M={gemm['M']}, N={gemm['N']}, K={gemm['K']}: the "
+                                        "step's largest lazy-update product)",
+                         "avg_launch_ms": gemm["ms"], "launches_timed": gemm["reps"]},
+            "roofline_syrk": {"bound": "tensor", "kernel": "syrk_bf16_tcgen05_kernel",
+                              "achieved": syrk_tflops, "peak": bf16, "unit": "TFLOP/s",
+                              "frac": syrk_tflops / bf16, "traffic": None,
+                              "peak_source": f"{peak_kind} bf16 burst",
+                              "frac_of_sustained": syrk_tflops / bf16_sus,
+                              "algorithmic": f"d(d+1)N = {syrk_flops:.4g} flop per launch"},
+            "stages": stages,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": statistics.mean(e2e_ms)},
-            "gpu_launches": launches_per_step(d, q) * args.steps,
+            "gpu_launches": (launches * args.steps) if launches is not None else None,
+            "gpu_launches_per_step": launches,
             "execution": "eager C ABI calls" if args.eager else
                          "CUDA graphs recorded from the C ABI calls, replayed",
             "clocks": clk.summary(),
@@ -563,6 +670,7 @@ def run_ours(args):
 
 def main():
     args = parse_args()
+    args.e2e_steps = max(1, args.e2e_steps)
     if args.impl == "reference":
         run_reference(args)
     else:

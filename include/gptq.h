@@ -6,8 +6,11 @@
  *   gptq_prepare_hinv        dead columns, damping, act-order, U = upper Cholesky factor of H^-1
  *   gptq_quantize_layer      column sweep with OBS compensation and lazy block updates
  *   gptq_pack                codes -> packed int words, scales/zeros -> fp16
+ *   gptq_quantize_pack_layer the sweep writing the packed words and fp16 scales/zeros directly
  *   rtn_quantize             round-to-nearest baseline with the same quantizer
  *   gptq_dequant_gemv        Y = X W_hat^T on the packed layer (batch 1 to 8), the format's consumer
+ *   gptq_gemm_f32            C = alpha op(A) op(B) + beta C at fp32 accuracy: the product kernel
+ *                            of prepare and of the lazy block update, exposed on its own
  *   gptq_quantize_layer_noalloc  gptq_quantize_layer on a fixed device scratch array
  *
  * Sources (page title, section):
@@ -197,6 +200,29 @@ int gptq_pack(const uint8_t* codes, int64_t d_out, int64_t d_in, int bits, const
               uint16_t* zeros_f16, gptq_stream_t stream);
 
 /*
+ * gptq_quantize_pack_layer — gptq_quantize_layer followed by gptq_pack in one pass: the sweep
+ * writes the packed layer directly, with no uint8 codes array and no separate pack step
+ * ([GPTQ-MATH] §2 Lazy Batch Updates for the sweep, §Inference Execution and Modern Kernel
+ * Architectures for the storage: eight 4-bit weights per int32 word).
+ *
+ * Same arguments and meaning as gptq_quantize_layer, except the outputs:
+ *   qweight      uint32 [d_out, d_in * bits / 32] device, 16-byte aligned: the words gptq_pack
+ *                would write from gptq_quantize_layer's codes, bit for bit.
+ *   scales_f16, zeros_f16  uint16 (fp16 bits) [d_out, n_groups] device: fp16 of scales/zeros
+ *                (round to nearest even), as gptq_pack writes them.
+ *   scales, zeros, g_idx   as in gptq_quantize_layer (fp32 parameters, sweep-group order).
+ * Natural order: each 32-code chunk of a row is packed in the sweep kernel as the chunk is
+ * finished. A permuted order: the sweep writes sweep-order codes into ws (gptq_workspace_size
+ * includes them) and one kernel gathers and packs them in the original column order.
+ */
+int gptq_quantize_pack_layer(const void* W, int w_dtype, int64_t ldw, int64_t d_out,
+                             int64_t d_in, const float* U, const int32_t* perm,
+                             const uint8_t* dead, const gptq_params* p, uint32_t* qweight,
+                             uint16_t* scales_f16, uint16_t* zeros_f16, float* scales,
+                             float* zeros, int32_t* g_idx, void* ws, size_t ws_bytes,
+                             int32_t* dev_status, gptq_stream_t stream);
+
+/*
  * rtn_quantize — round-to-nearest baseline ([GPTQ-MATH] §Comparison: RTN; [INT4-GPTQ] §Group
  * Quantization): (s, z) from the original W of each group (or row), then every weight
  * quantized independently with the same quantizer as gptq_quantize_layer, in natural column
@@ -264,6 +290,29 @@ int gptq_dequant_gemv(const uint32_t* qweight, int64_t d_out, int64_t d_in, int 
                       const uint16_t* scales_f16, const uint16_t* zeros_f16, int64_t n_groups,
                       int group_size, const int32_t* g_idx, const uint16_t* X, int64_t batch,
                       int64_t ldx, float* Y, int64_t ldy, gptq_stream_t stream);
+
+/*
+ * gptq_gemm_f32 — C = alpha * op(A) * op(B) + beta * C in fp32, the product that
+ * gptq_prepare_hinv and gptq_quantize_layer use for their block products: the lazy block
+ * update W[:, F] -= Err_B U[B, F] ([GPTQ-MATH] §2 Lazy Batch Updates) and the block steps of
+ * the Cholesky factor and its inverse (§3 Cholesky Decomposition and Pre-computation).
+ * Exposed so that the kernel can be checked and timed on its own.
+ *
+ * Large products run on the tcgen05 tensor cores with the three-term TF32 split
+ * (x = x_hi + x_lo, a b ~ a_hi b_hi + a_hi b_lo + a_lo b_hi), each accumulator covering a bounded
+ * stretch of K and the stretches summed in fp32; products up to 512^3 run on CUDA cores.
+ * Either way the result carries fp32-level accuracy (about 2^-21 relative per product).
+ *
+ *   All matrices row-major fp32, device pointers. op(A) is M x K: A[m*lda + k] when trans_a
+ *   is 0, A[k*lda + m] when 1; op(B) is K x N: B[k*ldb + n] when trans_b is 0, B[n*ldb + k]
+ *   when 1; C[m*ldc + n]. M, N >= 1, K >= 0 (K = 0 gives C = beta C); leading dimensions at
+ *   least the row length they index. beta == 0 means C is not read.
+ *   dev_status: as elsewhere (NULL allowed); the kernels do no work while it holds an error.
+ * Returns GPTQ_ERR_INVALID_ARG for a null pointer or an impossible shape.
+ */
+int gptq_gemm_f32(int64_t M, int64_t N, int64_t K, float alpha, const float* A, int64_t lda,
+                  int trans_a, const float* B, int64_t ldb, int trans_b, float beta, float* C,
+                  int64_t ldc, int32_t* dev_status, gptq_stream_t stream);
 
 #ifdef __cplusplus
 }

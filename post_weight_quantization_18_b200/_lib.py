@@ -32,7 +32,8 @@ GPTQ_ORDER_GIVEN = 2
 
 EXPORTED = ("gptq_workspace_size", "gptq_hessian_accumulate", "gptq_prepare_hinv",
             "gptq_quantize_layer", "gptq_pack", "rtn_quantize", "gptq_status_string",
-            "gptq_quantize_layer_noalloc", "gptq_dequant_gemv")
+            "gptq_quantize_layer_noalloc", "gptq_dequant_gemv", "gptq_gemm_f32",
+            "gptq_quantize_pack_layer")
 GPTQ_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -81,6 +82,11 @@ def _load() -> ctypes.CDLL:
     lib.rtn_quantize.restype = I32
     lib.gptq_dequant_gemv.argtypes = [P, I64, I64, I32, P, P, I64, I32, P, P, I64, I64, P, I64, P]
     lib.gptq_dequant_gemv.restype = I32
+    lib.gptq_gemm_f32.argtypes = [I64, I64, I64, F32, P, I64, I32, P, I64, I32, F32, P, I64, P, P]
+    lib.gptq_gemm_f32.restype = I32
+    lib.gptq_quantize_pack_layer.argtypes = [P, I32, I64, I64, I64, P, P, P, PP, P, P, P, P, P, P,
+                                             P, SZ, P, P]
+    lib.gptq_quantize_pack_layer.restype = I32
     lib.gptq_status_string.argtypes = [I32]
     lib.gptq_status_string.restype = ctypes.c_char_p
     return lib
@@ -283,3 +289,60 @@ def rtn_quantize(W: torch.Tensor, params: gptq_params, codes: torch.Tensor, scal
     rc = _lib.rtn_quantize(_ptr(W), _dtype_code(W), W.stride(0), n, d, ctypes.byref(params),
                            _ptr(codes), _ptr(scales), _ptr(zeros), _stream())
     _check(rc, "rtn_quantize")
+
+
+def gptq_gemm_f32(A: torch.Tensor, B: torch.Tensor, C: torch.Tensor, alpha: float = 1.0,
+                  beta: float = 0.0, trans_a: bool = False, trans_b: bool = False,
+                  dev_status: torch.Tensor | None = None) -> None:
+    """C = alpha op(A) op(B) + beta C (fp32, row-major tensors; op = transpose when trans_*)."""
+    for t, name in ((A, "A"), (B, "B"), (C, "C")):
+        _dev(t, name, torch.float32, 2)
+        _row_major(t, name)
+    M = A.shape[1] if trans_a else A.shape[0]
+    K = A.shape[0] if trans_a else A.shape[1]
+    Kb = B.shape[1] if trans_b else B.shape[0]
+    N = B.shape[0] if trans_b else B.shape[1]
+    if Kb != K or tuple(C.shape) != (M, N):
+        raise ValueError("shapes of A, B and C do not form a product")
+    rc = _lib.gptq_gemm_f32(M, N, K, float(alpha), _ptr(A), A.stride(0), int(bool(trans_a)),
+                            _ptr(B), B.stride(0), int(bool(trans_b)), float(beta), _ptr(C),
+                            C.stride(0), _ptr(dev_status), _stream())
+    _check(rc, "gptq_gemm_f32")
+
+
+def gptq_quantize_pack_layer(W: torch.Tensor, U: torch.Tensor, perm: torch.Tensor,
+                             dead: torch.Tensor, params: gptq_params, qweight: torch.Tensor,
+                             scales_f16: torch.Tensor, zeros_f16: torch.Tensor,
+                             scales: torch.Tensor, zeros: torch.Tensor, g_idx: torch.Tensor,
+                             ws: torch.Tensor, dev_status: torch.Tensor | None = None) -> None:
+    """The column sweep writing the packed layer directly (qweight int32/uint32 words, fp16 bits
+    of scales and zeros as int16 tensors), plus fp32 scales/zeros and g_idx."""
+    _dev(W, "W", None, 2)
+    _row_major(W, "W")
+    n, d = W.shape
+    _dev(U, "U", torch.float32, 2)
+    _dev(scales, "scales", torch.float32, 2)
+    _dev(zeros, "zeros", torch.float32, 2)
+    _dev(g_idx, "g_idx", torch.int32, 1)
+    _dev(ws, "ws")
+    for t, name in ((qweight, "qweight"), (scales_f16, "scales_f16"), (zeros_f16, "zeros_f16")):
+        _dev(t, name)
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    G = 1 if params.group_size == -1 else d // params.group_size
+    if qweight.element_size() != 4 or tuple(qweight.shape) != (n, d * params.bits // 32):
+        raise ValueError("qweight must be 32-bit words [d_out, d_in * bits / 32]")
+    for t in (scales, zeros, scales_f16, zeros_f16):
+        if tuple(t.shape) != (n, G) or not t.is_contiguous():
+            raise ValueError("scales / zeros (fp32 and fp16) must be contiguous [d_out, n_groups]")
+    if scales_f16.element_size() != 2 or zeros_f16.element_size() != 2:
+        raise ValueError("scales_f16 / zeros_f16 hold 16-bit patterns")
+    if U.shape != (d, d) or g_idx.numel() != d:
+        raise ValueError("U must be d_in x d_in and g_idx must have d_in entries")
+    rc = _lib.gptq_quantize_pack_layer(_ptr(W), _dtype_code(W), W.stride(0), n, d, _ptr(U),
+                                       _ptr(perm), _ptr(dead), ctypes.byref(params),
+                                       _ptr(qweight), _ptr(scales_f16), _ptr(zeros_f16),
+                                       _ptr(scales), _ptr(zeros), _ptr(g_idx), _ptr(ws),
+                                       ws.numel() * ws.element_size(), _ptr(dev_status),
+                                       _stream())
+    _check(rc, "gptq_quantize_pack_layer")

@@ -48,7 +48,7 @@ struct QuantWs {
   float* Wwork;
   float* Err;
   uint8_t* codes_sweep;
-  int32_t* inv_perm;  // static groups: the inverse column permutation
+  int32_t* inv_perm;  // static groups or a permuted order: the inverse column permutation
   size_t bytes;
 };
 
@@ -66,7 +66,7 @@ QuantWs quant_ws_layout(void* ws, int64_t n, int64_t d, int order, int static_gr
     off += align_up((size_t)n * d);
   }
   w.inv_perm = nullptr;
-  if (static_groups) {
+  if (static_groups || order != GPTQ_ORDER_NATURAL) {
     w.inv_perm = reinterpret_cast<int32_t*>(base + off);
     off += align_up((size_t)d * sizeof(int32_t));
   }
@@ -332,6 +332,9 @@ struct SweepCtx {
   int n, d, bits, g, sym;
   const int32_t* perm;  // static groups: the sweep order, for each column's original group
   int static_groups;
+  uint32_t* qweight;    // packed output in natural order (else null: uint8 codes)
+  uint16_t* s16;        // fp16 copies of the dynamic group parameters (packed output)
+  uint16_t* z16;
   int32_t* st;
   cudaStream_t s;
 };
@@ -340,7 +343,7 @@ int rec_sweep(const SweepCtx& c, int a, int b) {
   using namespace gptq_host;
   if (b - a <= 128)
     return sweep_block(c.Wwork, c.U, c.Err, c.codes, c.scales, c.zeros, c.n, c.d, a, c.bits, c.g,
-                       c.sym, c.perm, c.static_groups, c.st, c.s);
+                       c.sym, c.perm, c.static_groups, c.qweight, c.s16, c.z16, c.st, c.s);
   const int m = a + split_point(b - a);
   int rc;
   if ((rc = rec_sweep(c, a, m))) return rc;
@@ -349,6 +352,60 @@ int rec_sweep(const SweepCtx& c, int a, int b) {
                      c.d, false, 1.f, c.Wwork + m, c.d, false, c.st, c.s)))
     return rc;
   return rec_sweep(c, m, b);
+}
+
+// The rows of the sweep in two panels on two streams. Rows are independent given U
+// ([GPTQ-MATH] §The Layer-Wise Reconstruction Problem: the objective is a sum over rows), so
+// each panel runs its own block recursion; one panel's latency-bound 128-column sweeps then
+// share the SMs with the other panel's tensor-core lazy updates instead of leaving them idle.
+struct SweepStreams {
+  bool ready = false;
+  cudaStream_t side = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+
+SweepStreams* sweep_streams() {
+  thread_local SweepStreams per_device[kSideDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kSideDevices) return nullptr;
+  SweepStreams& ss = per_device[dev];
+  if (!ss.ready) {
+    if (cudaStreamCreateWithFlags(&ss.side, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess)
+      return nullptr;
+    ss.ready = true;
+  }
+  return &ss;
+}
+
+constexpr int kPanelMinRows = 1024;  // below this one panel (the leaves do not fill the GPU)
+
+int sweep_in_panels(const SweepCtx& c) {
+  const int n1 = ((c.n / 2 + 15) / 16) * 16;  // whole 16-row sweep CTAs in the first panel
+  if (c.n < kPanelMinRows || n1 >= c.n) return rec_sweep(c, 0, c.d);
+  SweepStreams* ss = sweep_streams();
+  if (ss == nullptr) return GPTQ_ERR_CUDA;
+  const long long G = (c.g > 0) ? c.d / c.g : 1;
+  SweepCtx c1 = c, c2 = c;
+  c1.n = n1;
+  c2.n = c.n - n1;
+  c2.Wwork += (long long)n1 * c.d;
+  c2.Err += (long long)n1 * c.d;
+  c2.codes += (long long)n1 * c.d;
+  c2.scales += n1 * G;
+  c2.zeros += n1 * G;
+  if (c.qweight != nullptr) c2.qweight += (long long)n1 * (c.d / 32) * c.bits;
+  if (c.s16 != nullptr) {
+    c2.s16 += n1 * G;
+    c2.z16 += n1 * G;
+  }
+  c2.s = ss->side;
+  int rc;
+  if ((rc = ev_rec(ss->fork, c.s)) || (rc = ev_wait(ss->side, ss->fork))) return rc;
+  if ((rc = rec_sweep(c1, 0, c.d)) || (rc = rec_sweep(c2, 0, c.d))) return rc;
+  if ((rc = ev_rec(ss->join, ss->side)) || (rc = ev_wait(c.s, ss->join))) return rc;
+  return 0;
 }
 
 }  // namespace
@@ -421,15 +478,67 @@ int gptq_prepare_hinv(float* H, int64_t d_in, const gptq_params* p, float* U, in
   using namespace gptq_host;
   int rc = 0;
   if (p->order == GPTQ_ORDER_NATURAL) {
-    rc = prep_identity_perm(perm, d, s);
+    rc = prep_identity_perm(perm, d, dev_status, s);
   } else {
-    if (p->order == GPTQ_ORDER_DESC_ACT) rc = prep_act_order(H, perm, d, s);
-    if (!rc) rc = prep_permute_sym(H, U, perm, d, s);
-    if (!rc) rc = prep_copy_upper(U, H, d, s);
+    if (p->order == GPTQ_ORDER_DESC_ACT) rc = prep_act_order(H, perm, d, dev_status, s);
+    if (!rc) rc = prep_permute_sym(H, U, perm, d, dev_status, s);
+    if (!rc) rc = prep_copy_upper(U, H, d, dev_status, s);
   }
   if (!rc) rc = prep_dead_damp(H, dead, d, p->percdamp, dev_status, s);
-  if (!rc) rc = prep_zero_lower(U, d, s);
+  if (!rc) rc = prep_zero_lower(U, d, dev_status, s);
   if (!rc) rc = rec_prepare(H, U, d, 0, d, 0, prep_streams(), dev_status, s);
+  return rc ? GPTQ_ERR_CUDA : GPTQ_OK;
+}
+
+// Shared by gptq_quantize_layer (codes != null: uint8 codes) and gptq_quantize_pack_layer
+// (qweight != null: packed words and fp16 parameters, no codes array).
+static int quantize_impl(const void* W, int w_dtype, int64_t ldw, int64_t d_out, int64_t d_in,
+                         const float* U, const int32_t* perm, const uint8_t* dead,
+                         const gptq_params* p, uint8_t* codes, uint32_t* qweight,
+                         uint16_t* scales_f16, uint16_t* zeros_f16, float* scales, float* zeros,
+                         int32_t* g_idx, void* ws, size_t ws_bytes, int32_t* dev_status,
+                         gptq_stream_t stream) {
+  if (!params_ok(p) || W == nullptr || U == nullptr || perm == nullptr || dead == nullptr ||
+      scales == nullptr || zeros == nullptr || g_idx == nullptr || ws == nullptr)
+    return GPTQ_ERR_INVALID_ARG;
+  if (d_out < 1 || d_in < 128 || d_in % 128 != 0 || ldw < d_in || d_in > (1 << 30) ||
+      d_out > (1 << 30))
+    return GPTQ_ERR_INVALID_ARG;
+  if (w_dtype != GPTQ_BF16 && w_dtype != GPTQ_F32) return GPTQ_ERR_UNSUPPORTED;
+  if (!aligned(U, 16) || !aligned(ws, 16)) return GPTQ_ERR_INVALID_ARG;
+  if (codes != nullptr && !aligned(codes, 4)) return GPTQ_ERR_INVALID_ARG;
+  if (qweight != nullptr && !aligned(qweight, 16)) return GPTQ_ERR_INVALID_ARG;
+  const QuantWs w = quant_ws_layout(ws, d_out, d_in, p->order, p->static_groups);
+  if (ws_bytes < w.bytes) return GPTQ_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int n = (int)d_out, d = (int)d_in;
+  const bool natural = p->order == GPTQ_ORDER_NATURAL;
+  using namespace gptq_host;
+  int rc = sweep_gather_w(W, w_dtype, ldw, n, d, perm, dead, w.Wwork, dev_status, s);
+  if (!rc && w.inv_perm != nullptr) rc = sweep_invert_perm(perm, w.inv_perm, d, dev_status, s);
+  if (!rc && p->group_size == -1)
+    rc = sweep_row_params(w.Wwork, n, d, p->bits, p->sym, scales, zeros, scales_f16, zeros_f16,
+                          dev_status, s);
+  if (!rc && p->static_groups)
+    rc = sweep_static_params(w.Wwork, w.inv_perm, n, d, p->group_size, p->bits, p->sym, scales,
+                             zeros, scales_f16, zeros_f16, dev_status, s);
+  // Natural order: the sweep writes the output (codes, or packed words) directly; a permuted
+  // order sweeps into sweep-order codes that are then unpermuted (and packed).
+  uint8_t* cs = natural ? codes : w.codes_sweep;
+  uint32_t* qw_sweep = natural ? qweight : nullptr;
+  const bool dyn = p->group_size > 0 && !p->static_groups;  // parameters decided by the sweep
+  SweepCtx c{w.Wwork, U, w.Err, cs, scales, zeros, n, d, p->bits, p->group_size, p->sym,
+             perm, p->static_groups, qw_sweep, dyn ? scales_f16 : nullptr,
+             dyn ? zeros_f16 : nullptr, dev_status, s};
+  if (!rc) rc = sweep_in_panels(c);
+  if (!rc && !natural) {
+    if (qweight != nullptr)
+      rc = sweep_unpermute_pack(cs, w.inv_perm, n, d, p->bits, qweight, dev_status, s);
+    else
+      rc = sweep_unpermute_codes(cs, perm, codes, n, d, dev_status, s);
+  }
+  if (!rc)
+    rc = sweep_g_idx(p->static_groups ? nullptr : perm, g_idx, d, p->group_size, dev_status, s);
   return rc ? GPTQ_ERR_CUDA : GPTQ_OK;
 }
 
@@ -438,34 +547,22 @@ int gptq_quantize_layer(const void* W, int w_dtype, int64_t ldw, int64_t d_out, 
                         const gptq_params* p, uint8_t* codes, float* scales, float* zeros,
                         int32_t* g_idx, void* ws, size_t ws_bytes, int32_t* dev_status,
                         gptq_stream_t stream) {
-  if (!params_ok(p) || W == nullptr || U == nullptr || perm == nullptr || dead == nullptr ||
-      codes == nullptr || scales == nullptr || zeros == nullptr || g_idx == nullptr ||
-      ws == nullptr)
+  if (codes == nullptr) return GPTQ_ERR_INVALID_ARG;
+  return quantize_impl(W, w_dtype, ldw, d_out, d_in, U, perm, dead, p, codes, nullptr, nullptr,
+                       nullptr, scales, zeros, g_idx, ws, ws_bytes, dev_status, stream);
+}
+
+int gptq_quantize_pack_layer(const void* W, int w_dtype, int64_t ldw, int64_t d_out,
+                             int64_t d_in, const float* U, const int32_t* perm,
+                             const uint8_t* dead, const gptq_params* p, uint32_t* qweight,
+                             uint16_t* scales_f16, uint16_t* zeros_f16, float* scales,
+                             float* zeros, int32_t* g_idx, void* ws, size_t ws_bytes,
+                             int32_t* dev_status, gptq_stream_t stream) {
+  if (qweight == nullptr || scales_f16 == nullptr || zeros_f16 == nullptr)
     return GPTQ_ERR_INVALID_ARG;
-  if (d_out < 1 || d_in < 128 || d_in % 128 != 0 || ldw < d_in || d_in > (1 << 30) ||
-      d_out > (1 << 30))
-    return GPTQ_ERR_INVALID_ARG;
-  if (w_dtype != GPTQ_BF16 && w_dtype != GPTQ_F32) return GPTQ_ERR_UNSUPPORTED;
-  if (!aligned(U, 16) || !aligned(codes, 4) || !aligned(ws, 16)) return GPTQ_ERR_INVALID_ARG;
-  const QuantWs w = quant_ws_layout(ws, d_out, d_in, p->order, p->static_groups);
-  if (ws_bytes < w.bytes) return GPTQ_ERR_WORKSPACE;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const int n = (int)d_out, d = (int)d_in;
-  using namespace gptq_host;
-  int rc = sweep_gather_w(W, w_dtype, ldw, n, d, perm, dead, w.Wwork, dev_status, s);
-  if (!rc && p->group_size == -1)
-    rc = sweep_row_params(w.Wwork, n, d, p->bits, p->sym, scales, zeros, dev_status, s);
-  if (!rc && p->static_groups)
-    rc = sweep_static_params(w.Wwork, perm, w.inv_perm, n, d, p->group_size, p->bits, p->sym,
-                             scales, zeros, dev_status, s);
-  uint8_t* cs = (p->order == GPTQ_ORDER_NATURAL) ? codes : w.codes_sweep;
-  SweepCtx c{w.Wwork, U, w.Err, cs, scales, zeros, n, d, p->bits, p->group_size, p->sym,
-             perm, p->static_groups, dev_status, s};
-  if (!rc) rc = rec_sweep(c, 0, d);
-  if (!rc && p->order != GPTQ_ORDER_NATURAL)
-    rc = sweep_unpermute_codes(cs, perm, codes, n, d, dev_status, s);
-  if (!rc) rc = sweep_g_idx(p->static_groups ? nullptr : perm, g_idx, d, p->group_size, s);
-  return rc ? GPTQ_ERR_CUDA : GPTQ_OK;
+  return quantize_impl(W, w_dtype, ldw, d_out, d_in, U, perm, dead, p, nullptr, qweight,
+                       scales_f16, zeros_f16, scales, zeros, g_idx, ws, ws_bytes, dev_status,
+                       stream);
 }
 
 int gptq_pack(const uint8_t* codes, int64_t d_out, int64_t d_in, int bits, const float* scales,
@@ -507,6 +604,30 @@ int gptq_dequant_gemv(const uint32_t* qweight, int64_t d_out, int64_t d_in, int 
   return gptq_host::dequant_gemv(qweight, (int)d_out, (int)d_in, bits, scales_f16, zeros_f16,
                                  (int)n_groups, g_idx ? 0 : group_size, g_idx, X, (int)batch, ldx,
                                  Y, ldy, reinterpret_cast<cudaStream_t>(stream))
+             ? GPTQ_ERR_CUDA
+             : GPTQ_OK;
+}
+
+int gptq_gemm_f32(int64_t M, int64_t N, int64_t K, float alpha, const float* A, int64_t lda,
+                  int trans_a, const float* B, int64_t ldb, int trans_b, float beta, float* C,
+                  int64_t ldc, int32_t* dev_status, gptq_stream_t stream) {
+  if (C == nullptr || M < 1 || N < 1 || K < 0 || M > (1 << 30) || N > (1 << 30) ||
+      K > (1 << 30) || (trans_a != 0 && trans_a != 1) || (trans_b != 0 && trans_b != 1))
+    return GPTQ_ERR_INVALID_ARG;
+  if (K > 0 && (A == nullptr || B == nullptr)) return GPTQ_ERR_INVALID_ARG;
+  const int64_t a_row = trans_a ? M : K, b_row = trans_b ? K : N;
+  if (ldc < N || (K > 0 && (lda < a_row || ldb < b_row))) return GPTQ_ERR_INVALID_ARG;
+  if (!aligned(C, 4) || (K > 0 && (!aligned(A, 4) || !aligned(B, 4))))
+    return GPTQ_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (K == 0) {  // C = beta C (alpha times an empty product)
+    return gptq_host::gemm_f32((int)M, (int)N, 0, 0.f, C, ldc, false, C, ldc, false, beta, C, ldc,
+                               false, dev_status, s)
+               ? GPTQ_ERR_CUDA
+               : GPTQ_OK;
+  }
+  return gptq_host::gemm_f32((int)M, (int)N, (int)K, alpha, A, lda, trans_a != 0, B, ldb,
+                             trans_b != 0, beta, C, ldc, false, dev_status, s)
              ? GPTQ_ERR_CUDA
              : GPTQ_OK;
 }

@@ -64,32 +64,47 @@ int gemm_tf32x3(int M, int N, int K, float alpha, const float* A, long long lda,
                 int tri = kTriNone, int max_ctas = 0);
 
 // ---- prepare ----
-int prep_permute_sym(const float* H, float* Hp, const int32_t* perm, int d, cudaStream_t stream);
-int prep_copy_upper(const float* src, float* dst, int d, cudaStream_t stream);
-int prep_act_order(const float* H, int32_t* perm, int d, cudaStream_t stream);
-int prep_identity_perm(int32_t* perm, int d, cudaStream_t stream);
+// Every kernel below, like all kernels given a status word, does no work while status[0] != 0.
+int prep_permute_sym(const float* H, float* Hp, const int32_t* perm, int d,
+                     const int32_t* status, cudaStream_t stream);
+int prep_copy_upper(const float* src, float* dst, int d, const int32_t* status,
+                    cudaStream_t stream);
+int prep_act_order(const float* H, int32_t* perm, int d, const int32_t* status,
+                   cudaStream_t stream);
+int prep_identity_perm(int32_t* perm, int d, const int32_t* status, cudaStream_t stream);
 int prep_dead_damp(float* H, uint8_t* dead, int d, float percdamp, int32_t* status,
                    cudaStream_t stream);
-int prep_zero_lower(float* U, int d, cudaStream_t stream);
+int prep_zero_lower(float* U, int d, const int32_t* status, cudaStream_t stream);
 int prep_base_block(float* Hblk, float* Ublk, int n, int ld, int index0, int32_t* status,
                     cudaStream_t stream);
 constexpr int kPrepBase = 128;
 
 // ---- sweep ----
+// qweight / s16 / z16 (packed output, gptq_quantize_pack_layer) may be null: then the sweep
+// writes uint8 codes and the fp32 parameters only.
 int sweep_gather_w(const void* W, int w_dtype, long long ldw, int n, int d, const int32_t* perm,
                    const uint8_t* dead, float* Wwork, const int32_t* status, cudaStream_t stream);
 int sweep_row_params(const float* Wwork, int n, int d, int bits, int sym, float* scales,
-                     float* zeros, const int32_t* status, cudaStream_t stream);
+                     float* zeros, uint16_t* s16, uint16_t* z16, const int32_t* status,
+                     cudaStream_t stream);
 int sweep_block(float* Wwork, const float* U, float* Err, uint8_t* codes, float* scales,
                 float* zeros, int n, int d, int col0, int bits, int group_size, int sym,
-                const int32_t* perm, int static_groups, int32_t* status, cudaStream_t stream);
-// Static groups: inv = perm^-1, then (s, z) [n, d / group_size] of the original-order groups.
-int sweep_static_params(const float* Wwork, const int32_t* perm, int32_t* inv, int n, int d,
-                        int group_size, int bits, int sym, float* scales, float* zeros,
-                        const int32_t* status, cudaStream_t stream);
+                const int32_t* perm, int static_groups, uint32_t* qweight, uint16_t* s16,
+                uint16_t* z16, int32_t* status, cudaStream_t stream);
+// inv = perm^-1.
+int sweep_invert_perm(const int32_t* perm, int32_t* inv, int d, const int32_t* status,
+                      cudaStream_t stream);
+// Static groups: (s, z) [n, d / group_size] of the original-order groups (inv = perm^-1).
+int sweep_static_params(const float* Wwork, const int32_t* inv, int n, int d, int group_size,
+                        int bits, int sym, float* scales, float* zeros, uint16_t* s16,
+                        uint16_t* z16, const int32_t* status, cudaStream_t stream);
 int sweep_unpermute_codes(const uint8_t* codes_sweep, const int32_t* perm, uint8_t* codes, int n,
                           int d, const int32_t* status, cudaStream_t stream);
-int sweep_g_idx(const int32_t* perm, int32_t* g_idx, int d, int group_size, cudaStream_t stream);
+// Sweep-order codes -> packed words in the original column order (inv = perm^-1).
+int sweep_unpermute_pack(const uint8_t* codes_sweep, const int32_t* inv, int n, int d, int bits,
+                         uint32_t* qweight, const int32_t* status, cudaStream_t stream);
+int sweep_g_idx(const int32_t* perm, int32_t* g_idx, int d, int group_size,
+                const int32_t* status, cudaStream_t stream);
 
 // ---- dequantizing matrix-vector product on the packed format ----
 int dequant_gemv(const uint32_t* qweight, int n, int d, int bits, const uint16_t* scales_f16,

@@ -23,7 +23,9 @@ namespace {
 // Hp[a][b] = H[pi a][pi b] on the upper triangle, reading H's upper triangle symmetrically:
 // rows on grid y, columns of the row's span strided over grid x (tri_fill.cuh).
 __global__ void permute_sym_kernel(const float* __restrict__ H, float* __restrict__ Hp,
-                                   const int32_t* __restrict__ perm, int d) {
+                                   const int32_t* __restrict__ perm, int d,
+                                   const int32_t* status) {
+  if (gptq::status_bad(status)) return;
   for (long long a = blockIdx.y; a < d; a += gridDim.y) {
     long long lo, hi;
     gptq::tri_row_span(gptq::kUpperWithDiag, a, d, lo, hi);
@@ -35,7 +37,9 @@ __global__ void permute_sym_kernel(const float* __restrict__ H, float* __restric
 }
 
 // dst's upper triangle (with the diagonal) = src's, same layout.
-__global__ void copy_upper_kernel(const float* __restrict__ src, float* __restrict__ dst, int d) {
+__global__ void copy_upper_kernel(const float* __restrict__ src, float* __restrict__ dst, int d,
+                                  const int32_t* status) {
+  if (gptq::status_bad(status)) return;
   for (long long a = blockIdx.y; a < d; a += gridDim.y) {
     long long lo, hi;
     gptq::tri_row_span(gptq::kUpperWithDiag, a, d, lo, hi);
@@ -48,8 +52,12 @@ __global__ void copy_upper_kernel(const float* __restrict__ src, float* __restri
 // Stable descending rank of diag(H): rank_i = #{j : h_j > h_i or (h_j == h_i and j < i)};
 // perm[rank_i] = i.
 __global__ void act_order_rank_kernel(const float* __restrict__ H, int32_t* __restrict__ perm,
-                                      int d) {
+                                      int d, const int32_t* status) {
   __shared__ float keys[1024];
+  __shared__ int bad;  // read once per block: every thread takes the same branch
+  if (threadIdx.x == 0) bad = gptq::status_bad(status) ? 1 : 0;
+  __syncthreads();
+  if (bad) return;
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   const float hi = (i < d) ? H[(long long)i * d + i] : 0.f;
   int rank = 0;
@@ -72,7 +80,8 @@ __global__ void act_order_rank_kernel(const float* __restrict__ H, int32_t* __re
   if (i < d) perm[rank] = i;
 }
 
-__global__ void identity_perm_kernel(int32_t* perm, int d) {
+__global__ void identity_perm_kernel(int32_t* perm, int d, const int32_t* status) {
+  if (gptq::status_bad(status)) return;
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < d; i += gridDim.x * blockDim.x)
     perm[i] = i;
 }
@@ -115,7 +124,8 @@ __global__ void dead_damp_kernel(float* __restrict__ H, uint8_t* __restrict__ de
 }
 
 // U's strictly lower triangle = 0: rows on grid y, columns strided over grid x (tri_fill.cuh).
-__global__ void zero_lower_kernel(float* U, int d) {
+__global__ void zero_lower_kernel(float* U, int d, const int32_t* status) {
+  if (gptq::status_bad(status)) return;
   for (long long r = blockIdx.y; r < d; r += gridDim.y) {
     long long lo, hi;
     gptq::tri_row_span(gptq::kStrictLower, r, d, lo, hi);
@@ -411,25 +421,28 @@ inline int grid_for(long long total) {
 
 namespace gptq_host {
 
-int prep_permute_sym(const float* H, float* Hp, const int32_t* perm, int d, cudaStream_t stream) {
+int prep_permute_sym(const float* H, float* Hp, const int32_t* perm, int d,
+                     const int32_t* status, cudaStream_t stream) {
   const dim3 grid((unsigned)((d + 1023) / 1024), (unsigned)(d < 65535 ? d : 65535));
-  permute_sym_kernel<<<grid, 256, 0, stream>>>(H, Hp, perm, d);
+  permute_sym_kernel<<<grid, 256, 0, stream>>>(H, Hp, perm, d, status);
   return cudaGetLastError() == cudaSuccess ? 0 : GPTQ_ERR_CUDA;
 }
 
-int prep_copy_upper(const float* src, float* dst, int d, cudaStream_t stream) {
+int prep_copy_upper(const float* src, float* dst, int d, const int32_t* status,
+                    cudaStream_t stream) {
   const dim3 grid((unsigned)((d + 1023) / 1024), (unsigned)(d < 65535 ? d : 65535));
-  copy_upper_kernel<<<grid, 256, 0, stream>>>(src, dst, d);
+  copy_upper_kernel<<<grid, 256, 0, stream>>>(src, dst, d, status);
   return cudaGetLastError() == cudaSuccess ? 0 : GPTQ_ERR_CUDA;
 }
 
-int prep_act_order(const float* H, int32_t* perm, int d, cudaStream_t stream) {
-  act_order_rank_kernel<<<(d + 255) / 256, 256, 0, stream>>>(H, perm, d);
+int prep_act_order(const float* H, int32_t* perm, int d, const int32_t* status,
+                   cudaStream_t stream) {
+  act_order_rank_kernel<<<(d + 255) / 256, 256, 0, stream>>>(H, perm, d, status);
   return cudaGetLastError() == cudaSuccess ? 0 : GPTQ_ERR_CUDA;
 }
 
-int prep_identity_perm(int32_t* perm, int d, cudaStream_t stream) {
-  identity_perm_kernel<<<grid_for(d), 256, 0, stream>>>(perm, d);
+int prep_identity_perm(int32_t* perm, int d, const int32_t* status, cudaStream_t stream) {
+  identity_perm_kernel<<<grid_for(d), 256, 0, stream>>>(perm, d, status);
   return cudaGetLastError() == cudaSuccess ? 0 : GPTQ_ERR_CUDA;
 }
 
@@ -439,9 +452,9 @@ int prep_dead_damp(float* H, uint8_t* dead, int d, float percdamp, int32_t* stat
   return cudaGetLastError() == cudaSuccess ? 0 : GPTQ_ERR_CUDA;
 }
 
-int prep_zero_lower(float* U, int d, cudaStream_t stream) {
+int prep_zero_lower(float* U, int d, const int32_t* status, cudaStream_t stream) {
   const dim3 grid((unsigned)((d + 1023) / 1024), (unsigned)(d < 65535 ? d : 65535));
-  zero_lower_kernel<<<grid, 256, 0, stream>>>(U, d);
+  zero_lower_kernel<<<grid, 256, 0, stream>>>(U, d, status);
   return cudaGetLastError() == cudaSuccess ? 0 : GPTQ_ERR_CUDA;
 }
 

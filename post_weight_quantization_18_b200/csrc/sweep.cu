@@ -23,9 +23,11 @@
 #include <float.h>
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "common.cuh"
 #include "gather4.cuh"
+#include "pack32.cuh"
 #include "kernels.h"
 #include "tri_fill.cuh"
 
@@ -76,14 +78,41 @@ __device__ __forceinline__ float group8_max(float v) {
   return fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
 }
 
+// 32 codes (c[i]: codes 4i .. 4i+3 as bytes) -> `bits` words of the packed row at out, the
+// layout of gptq_pack (pack32.cuh). out is aligned for the vector store of each width: the row
+// stride d * bits / 32 words and the chunk offset are multiples of it, qweight 16-byte aligned.
+__device__ __forceinline__ void store_packed_chunk(const uint32_t (&c)[8], int bits,
+                                                   uint32_t* out) {
+  if (bits == 4) {
+    uint32_t w[4];
+    gptq::pack32<4>(c, w);
+    *reinterpret_cast<uint4*>(out) = make_uint4(w[0], w[1], w[2], w[3]);
+  } else if (bits == 3) {
+    uint32_t w[3];
+    gptq::pack32<3>(c, w);
+    out[0] = w[0]; out[1] = w[1]; out[2] = w[2];
+  } else if (bits == 2) {
+    uint32_t w[2];
+    gptq::pack32<2>(c, w);
+    *reinterpret_cast<uint2*>(out) = make_uint2(w[0], w[1]);
+  } else {
+    uint32_t w[8];
+    gptq::pack32<8>(c, w);
+    reinterpret_cast<uint4*>(out)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    reinterpret_cast<uint4*>(out)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  }
+}
+
 // STATIC: static groups (one instance each, so the default path carries no extra branch).
-template <bool STATIC>
+// FINE: groups shorter than 32 columns, whose starts fall inside a 32-column chunk.
+template <bool STATIC, bool FINE>
 __global__ void __launch_bounds__(128)
 sweep_block_kernel(const __grid_constant__ CUtensorMap tmap_u, const float* __restrict__ Wwork,
                    float* __restrict__ Err, uint8_t* __restrict__ codes,
                    float* __restrict__ scales, float* __restrict__ zeros, int n, int d, int col0,
                    int bits, int g, int sym, const int32_t* __restrict__ perm,
-                   int32_t* status) {
+                   uint32_t* __restrict__ qweight, uint16_t* __restrict__ s16,
+                   uint16_t* __restrict__ z16, int32_t* status) {
   extern __shared__ __align__(128) float sw_smem[];
   float* Us = sw_smem;                // [128][128], zero below the diagonal
   float* invd = sw_smem + BLK * BLK;  // [128]
@@ -148,7 +177,10 @@ sweep_block_kernel(const __grid_constant__ CUtensorMap tmap_u, const float* __re
   const int gmask = grouped ? g - 1 : 0;
   const bool landed = gptq::mbar_wait(bar, 0, &abort_flag);
   if (!__syncthreads_and(landed)) {  // the copy did not arrive in time: report, touch nothing
-    if (tid == 0) gptq::set_status(status, GPTQ_ERR_TIMEOUT, 3);
+    if (tid == 0) {
+      gptq::set_status(status, GPTQ_ERR_TIMEOUT, 3);
+      gptq::mbar_drain(bar, 0);  // the CTA stays until the copy lands (bounded)
+    }
     return;
   }
   for (int t = tid; t < BLK; t += blockDim.x) invd[t] = __fdiv_rn(1.0f, Us[t * BLK + t]);
@@ -158,9 +190,46 @@ sweep_block_kernel(const __grid_constant__ CUtensorMap tmap_u, const float* __re
   uint8_t* crow = codes + (long long)rsafe * d + col0;
   const bool codes_vec = (reinterpret_cast<uintptr_t>(codes) & 3) == 0 && (d & 3) == 0;
   bool finite = true;
+  // (s, z) of the group that starts at block column j, from the current values of its g
+  // columns (min / max over the row's eight lanes).
+  auto group_params = [&](int j) {
+    float a = sym ? 0.f : FLT_MAX, b = -FLT_MAX;
+#pragma unroll
+    for (int c2 = 0; c2 < 4; ++c2)
+#pragma unroll
+      for (int e2 = 0; e2 < 4; ++e2) {
+        const int k = 32 * c2 + 4 * sub + e2;
+        const float v = w[4 * c2 + e2];
+        if (k >= j && k < j + g) {
+          if (sym) a = fmaxf(a, fabsf(v));
+          else { a = fminf(a, v); b = fmaxf(b, v); }
+        }
+      }
+    if (sym) {
+      a = group8_max(a);
+      sym_params(a, bits, s, z);
+    } else {
+      a = group8_min(a);
+      b = group8_max(b);
+      asym_params(a, b, maxq, s, z);
+    }
+    rs = __frcp_rn(s);
+    if (sub == 0 && live) {
+      const long long gi = (long long)row * G + (col0 + j) / g;
+      scales[gi] = s;
+      zeros[gi] = z;
+      if (s16 != nullptr) {  // packed output: the fp16 copies (round to nearest even)
+        s16[gi] = __half_as_ushort(__float2half_rn(s));
+        z16[gi] = __half_as_ushort(__float2half_rn(z));
+      }
+    }
+  };
 #pragma unroll
   for (int c = 0; c < 4; ++c) {                  // 32-column chunks
     float qk[4], ek[4];                          // this lane's four codes and errors of chunk c
+    // Groups of 32 columns or more start at chunk starts: their statistics are taken here,
+    // outside the column loop (which keeps that loop's unrolled code small).
+    if (!FINE && grouped && ((32 * c) & gmask) == 0) group_params(32 * c);
 #pragma unroll 1
     for (int so = 0; so < 8; ++so) {             // owner sub-lane within the chunk
 #pragma unroll
@@ -170,33 +239,8 @@ sweep_block_kernel(const __grid_constant__ CUtensorMap tmap_u, const float* __re
           s = stab[rl * BLK + j];
           rs = stab[16 * BLK + rl * BLK + j];
           z = stab[32 * BLK + rl * BLK + j];
-        } else if (grouped && (j & gmask) == 0) {
-          float a = sym ? 0.f : FLT_MAX, b = -FLT_MAX;
-#pragma unroll
-          for (int c2 = 0; c2 < 4; ++c2)
-#pragma unroll
-            for (int e2 = 0; e2 < 4; ++e2) {
-              const int k = 32 * c2 + 4 * sub + e2;
-              const float v = w[4 * c2 + e2];
-              if (k >= j && k < j + g) {
-                if (sym) a = fmaxf(a, fabsf(v));
-                else { a = fminf(a, v); b = fmaxf(b, v); }
-              }
-            }
-          if (sym) {
-            a = group8_max(a);
-            sym_params(a, bits, s, z);
-          } else {
-            a = group8_min(a);
-            b = group8_max(b);
-            asym_params(a, b, maxq, s, z);
-          }
-          rs = __frcp_rn(s);
-          if (sub == 0 && live) {
-            const long long gi = (long long)row * G + (col0 + j) / g;
-            scales[gi] = s;
-            zeros[gi] = z;
-          }
+        } else if (FINE && (j & gmask) == 0) {
+          group_params(j);
         }
         const float wj = __shfl_sync(0xffffffffu, w[4 * c + e], grp | so);
         const float qv = quant_code_rcp(wj, s, rs, z, maxq);
@@ -222,8 +266,20 @@ sweep_block_kernel(const __grid_constant__ CUtensorMap tmap_u, const float* __re
     if (live) {
       const int k0 = 32 * c + 4 * sub;
       *reinterpret_cast<float4*>(erow + k0) = make_float4(ek[0], ek[1], ek[2], ek[3]);
-      const uint32_t packed = (uint32_t)qk[0] | ((uint32_t)qk[1] << 8) |
-                              ((uint32_t)qk[2] << 16) | ((uint32_t)qk[3] << 24);
+    }
+    const uint32_t packed = (uint32_t)qk[0] | ((uint32_t)qk[1] << 8) | ((uint32_t)qk[2] << 16) |
+                            ((uint32_t)qk[3] << 24);
+    if (qweight != nullptr) {
+      // Packed output: the row's 32 codes of this chunk (four per lane) gathered in every lane
+      // of the row's group, packed by its first lane into `bits` words of the row's bit stream.
+      uint32_t cw[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) cw[k] = __shfl_sync(0xffffffffu, packed, grp | k);
+      if (sub == 0 && live)
+        store_packed_chunk(cw, bits, qweight + (long long)row * (d / 32) * bits +
+                                         (long long)(col0 / 32 + c) * bits);
+    } else if (live) {
+      const int k0 = 32 * c + 4 * sub;
       if (codes_vec) {
         *reinterpret_cast<uint32_t*>(crow + k0) = packed;
       } else {
@@ -258,7 +314,8 @@ __global__ void gather_w_kernel(const T* __restrict__ W, long long ldw, int n, i
 // One (s, z) per row from the whole row at the start of the sweep (group_size = -1).
 __global__ void row_params_kernel(const float* __restrict__ Wwork, int n, int d, int bits,
                                   int sym, float* __restrict__ scales,
-                                  float* __restrict__ zeros, const int32_t* status) {
+                                  float* __restrict__ zeros, uint16_t* __restrict__ s16,
+                                  uint16_t* __restrict__ z16, const int32_t* status) {
   if (gptq::status_bad(status)) return;
   const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -282,6 +339,10 @@ __global__ void row_params_kernel(const float* __restrict__ Wwork, int n, int d,
     else asym_params(mn, mx, (float)((1 << bits) - 1), s, z);
     scales[r] = s;
     zeros[r] = z;
+    if (s16 != nullptr) {
+      s16[r] = __half_as_ushort(__float2half_rn(s));
+      z16[r] = __half_as_ushort(__float2half_rn(z));
+    }
   }
 }
 
@@ -300,16 +361,44 @@ __global__ void unpermute_codes_kernel(const uint8_t* __restrict__ cs,
   }
 }
 
+// Permuted column order, packed output: one thread per (row, chunk of 32 original columns)
+// gathers its codes from the sweep-order codes (original column c sits at sweep position
+// inv[c]) and packs them into `bits` words (pack32.cuh). d is a multiple of 128.
+template <int BITS>
+__global__ void unpermute_pack_kernel(const uint8_t* __restrict__ cs,
+                                      const int32_t* __restrict__ inv, int n, int d,
+                                      uint32_t* __restrict__ qweight, const int32_t* status) {
+  if (gptq::status_bad(status)) return;
+  const int chunks = d / 32;
+  for (long long item = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+       item < (long long)n * chunks; item += (long long)gridDim.x * blockDim.x) {
+    const long long r = item / chunks;
+    const int ch = (int)(item % chunks);
+    const uint8_t* row = cs + r * d;
+    uint32_t c[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      uint32_t v = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) v |= (uint32_t)row[inv[ch * 32 + 4 * i + e]] << (8 * e);
+      c[i] = v;
+    }
+    store_packed_chunk(c, BITS, qweight + r * chunks * BITS + (long long)ch * BITS);
+  }
+}
+
 // g_idx[perm[k]] = k / g (groups in sweep order); perm == nullptr: g_idx[k] = k / g.
 __global__ void g_idx_kernel(const int32_t* __restrict__ perm, int32_t* __restrict__ g_idx, int d,
-                             int g) {
+                             int g, const int32_t* status) {
+  if (gptq::status_bad(status)) return;
   for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < d; k += gridDim.x * blockDim.x)
     g_idx[perm ? perm[k] : k] = (g > 0) ? k / g : 0;
 }
 
 // inv[perm[j]] = j.
 __global__ void invert_perm_kernel(const int32_t* __restrict__ perm, int32_t* __restrict__ inv,
-                                   int d) {
+                                   int d, const int32_t* status) {
+  if (gptq::status_bad(status)) return;
   for (int j = blockIdx.x * blockDim.x + threadIdx.x; j < d; j += gridDim.x * blockDim.x)
     inv[perm[j]] = j;
 }
@@ -320,7 +409,8 @@ __global__ void invert_perm_kernel(const int32_t* __restrict__ perm, int32_t* __
 __global__ void static_params_kernel(const float* __restrict__ Wwork,
                                      const int32_t* __restrict__ inv, int n, int d, int g,
                                      int bits, int sym, float* __restrict__ scales,
-                                     float* __restrict__ zeros, const int32_t* status) {
+                                     float* __restrict__ zeros, uint16_t* __restrict__ s16,
+                                     uint16_t* __restrict__ z16, const int32_t* status) {
   if (gptq::status_bad(status)) return;
   const int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -348,6 +438,10 @@ __global__ void static_params_kernel(const float* __restrict__ Wwork,
       else asym_params(mn, mx, maxq, sv, zv);
       scales[(long long)r * G + q] = sv;
       zeros[(long long)r * G + q] = zv;
+      if (s16 != nullptr) {
+        s16[(long long)r * G + q] = __half_as_ushort(__float2half_rn(sv));
+        z16[(long long)r * G + q] = __half_as_ushort(__float2half_rn(zv));
+      }
     }
   }
 }
@@ -378,17 +472,23 @@ int sweep_gather_w(const void* W, int w_dtype, long long ldw, int n, int d, cons
 }
 
 int sweep_row_params(const float* Wwork, int n, int d, int bits, int sym, float* scales,
-                     float* zeros, const int32_t* status, cudaStream_t stream) {
-  row_params_kernel<<<(n + 7) / 8, 256, 0, stream>>>(Wwork, n, d, bits, sym, scales, zeros,
-                                                     status);
+                     float* zeros, uint16_t* s16, uint16_t* z16, const int32_t* status,
+                     cudaStream_t stream) {
+  row_params_kernel<<<(n + 7) / 8, 256, 0, stream>>>(Wwork, n, d, bits, sym, scales, zeros, s16,
+                                                     z16, status);
   return cudaGetLastError() == cudaSuccess ? 0 : GPTQ_ERR_CUDA;
 }
 
 int sweep_block(float* Wwork, const float* U, float* Err, uint8_t* codes, float* scales,
                 float* zeros, int n, int d, int col0, int bits, int group_size, int sym,
-                const int32_t* perm, int static_groups, int32_t* status, cudaStream_t stream) {
-  if (ensure_smem_attr(reinterpret_cast<const void*>(sweep_block_kernel<false>), SW_SMEM) != 0 ||
-      ensure_smem_attr(reinterpret_cast<const void*>(sweep_block_kernel<true>), SW_SMEM_STATIC) != 0)
+                const int32_t* perm, int static_groups, uint32_t* qweight, uint16_t* s16,
+                uint16_t* z16, int32_t* status, cudaStream_t stream) {
+  if (ensure_smem_attr(reinterpret_cast<const void*>(sweep_block_kernel<false, false>), SW_SMEM) !=
+          0 ||
+      ensure_smem_attr(reinterpret_cast<const void*>(sweep_block_kernel<false, true>), SW_SMEM) !=
+          0 ||
+      ensure_smem_attr(reinterpret_cast<const void*>(sweep_block_kernel<true, false>),
+                       SW_SMEM_STATIC) != 0)
     return GPTQ_ERR_CUDA;
   CUtensorMap tu;  // the whole U (d x d fp32), copied 128 x 128 at a time without swizzle
   if (make_tmap_2d(&tu, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, U, (uint64_t)d, (uint64_t)d,
@@ -397,11 +497,17 @@ int sweep_block(float* Wwork, const float* U, float* Err, uint8_t* codes, float*
   const int warps_total = (n + ROWS_PER_WARP - 1) / ROWS_PER_WARP;
   const int grid = (warps_total + 3) / 4;  // 4 warps (16 rows) per CTA
   if (static_groups)
-    sweep_block_kernel<true><<<grid, 128, SW_SMEM_STATIC, stream>>>(
-        tu, Wwork, Err, codes, scales, zeros, n, d, col0, bits, group_size, sym, perm, status);
+    sweep_block_kernel<true, false><<<grid, 128, SW_SMEM_STATIC, stream>>>(
+        tu, Wwork, Err, codes, scales, zeros, n, d, col0, bits, group_size, sym, perm, qweight,
+        s16, z16, status);
+  else if (group_size > 0 && group_size < 32)
+    sweep_block_kernel<false, true><<<grid, 128, SW_SMEM, stream>>>(
+        tu, Wwork, Err, codes, scales, zeros, n, d, col0, bits, group_size, sym, perm, qweight,
+        s16, z16, status);
   else
-    sweep_block_kernel<false><<<grid, 128, SW_SMEM, stream>>>(
-        tu, Wwork, Err, codes, scales, zeros, n, d, col0, bits, group_size, sym, perm, status);
+    sweep_block_kernel<false, false><<<grid, 128, SW_SMEM, stream>>>(
+        tu, Wwork, Err, codes, scales, zeros, n, d, col0, bits, group_size, sym, perm, qweight,
+        s16, z16, status);
   return cudaGetLastError() == cudaSuccess ? 0 : GPTQ_ERR_CUDA;
 }
 
@@ -412,18 +518,38 @@ int sweep_unpermute_codes(const uint8_t* codes_sweep, const int32_t* perm, uint8
   return cudaGetLastError() == cudaSuccess ? 0 : GPTQ_ERR_CUDA;
 }
 
-int sweep_static_params(const float* Wwork, const int32_t* perm, int32_t* inv, int n, int d,
-                        int group_size, int bits, int sym, float* scales, float* zeros,
-                        const int32_t* status, cudaStream_t stream) {
-  invert_perm_kernel<<<grid_for(d), 256, 0, stream>>>(perm, inv, d);
-  if (cudaGetLastError() != cudaSuccess) return GPTQ_ERR_CUDA;
-  static_params_kernel<<<(n + 7) / 8, 256, 0, stream>>>(Wwork, inv, n, d, group_size, bits, sym,
-                                                         scales, zeros, status);
+int sweep_invert_perm(const int32_t* perm, int32_t* inv, int d, const int32_t* status,
+                      cudaStream_t stream) {
+  invert_perm_kernel<<<grid_for(d), 256, 0, stream>>>(perm, inv, d, status);
   return cudaGetLastError() == cudaSuccess ? 0 : GPTQ_ERR_CUDA;
 }
 
-int sweep_g_idx(const int32_t* perm, int32_t* g_idx, int d, int group_size, cudaStream_t stream) {
-  g_idx_kernel<<<grid_for(d), 256, 0, stream>>>(perm, g_idx, d, group_size);
+int sweep_static_params(const float* Wwork, const int32_t* inv, int n, int d, int group_size,
+                        int bits, int sym, float* scales, float* zeros, uint16_t* s16,
+                        uint16_t* z16, const int32_t* status, cudaStream_t stream) {
+  static_params_kernel<<<(n + 7) / 8, 256, 0, stream>>>(Wwork, inv, n, d, group_size, bits, sym,
+                                                         scales, zeros, s16, z16, status);
+  return cudaGetLastError() == cudaSuccess ? 0 : GPTQ_ERR_CUDA;
+}
+
+int sweep_unpermute_pack(const uint8_t* codes_sweep, const int32_t* inv, int n, int d, int bits,
+                         uint32_t* qweight, const int32_t* status, cudaStream_t stream) {
+  const long long items = (long long)n * (d / 32);
+  const int grid = grid_for(items);
+  if (bits == 2)
+    unpermute_pack_kernel<2><<<grid, 256, 0, stream>>>(codes_sweep, inv, n, d, qweight, status);
+  else if (bits == 3)
+    unpermute_pack_kernel<3><<<grid, 256, 0, stream>>>(codes_sweep, inv, n, d, qweight, status);
+  else if (bits == 4)
+    unpermute_pack_kernel<4><<<grid, 256, 0, stream>>>(codes_sweep, inv, n, d, qweight, status);
+  else
+    unpermute_pack_kernel<8><<<grid, 256, 0, stream>>>(codes_sweep, inv, n, d, qweight, status);
+  return cudaGetLastError() == cudaSuccess ? 0 : GPTQ_ERR_CUDA;
+}
+
+int sweep_g_idx(const int32_t* perm, int32_t* g_idx, int d, int group_size,
+                const int32_t* status, cudaStream_t stream) {
+  g_idx_kernel<<<grid_for(d), 256, 0, stream>>>(perm, g_idx, d, group_size, status);
   return cudaGetLastError() == cudaSuccess ? 0 : GPTQ_ERR_CUDA;
 }
 

@@ -8,8 +8,9 @@
 // Design (one CTA per SM, persistent):
 //   * Work unit = (256 x 256 output tile with i-block <= j-block, token chunk). Only tiles on or
 //     above the diagonal are scheduled; the token range is split into chunks of at most 8192
-//     tokens (and further only when the tiles alone cannot fill the SMs). Units are chunk-major
-//     so concurrently running CTAs share one L2-resident chunk of X.
+//     tokens (and further only when the tiles alone cannot fill the SMs). Units are ordered by
+//     groups of tiles, token range by token range inside a group, so that the CTAs running
+//     together share the L2-resident panels of X of one group and one range (syrk_units.cuh).
 //   * warp 0: TMA producer — per 64-token k-block, four 64x64 boxes of X for the A tile (rows
 //     i0..i0+255) and four for the B tile (j0..j0+255), 128-byte swizzled, 3-stage ring.
 //   * warp 1: TMEM owner and MMA issuer — per 16-token step two tcgen05.mma kind::f16 of
@@ -22,9 +23,13 @@
 //     (cp.reduce.async.bulk.tensor .add), which also clips the ragged edge of H. The MMA warp
 //     starts the next unit once both halves are drained.
 //   * Every mbarrier wait is bounded; on timeout the CTA records GPTQ_ERR_TIMEOUT, leaves its
-//     loops, frees TMEM and returns.
+//     loops, waits (bounded) for the loads and MMAs it already issued, frees TMEM and returns.
+#include <math.h>
+
 #include "common.cuh"
 #include "kernels.h"
+#include "syrk_units.cuh"
+#include "tri_fill.cuh"
 
 namespace {
 
@@ -45,22 +50,12 @@ constexpr uint32_t TMEM_COLS = 512;               // the two 128 x 256 halves of
 constexpr uint32_t IDESC = gptq::instr_desc(/*bf16*/ 1, /*A MN*/ 1, /*B MN*/ 1, MMA_M, BN);
 
 struct SyrkArgs {
-  int d, n_ib, n_jb, n_tiles, n_split, kb_per_split, nkb_total;
+  int d, n_tb, n_tiles, n_split, kb_per_split, nkb_total;
+  int grp;  // tile rows / columns per group (syrk_units.cuh)
   long long n_units;
   float alpha;
   int32_t* status;
 };
-
-// Tile t (0..n_tiles-1) -> (ib, jb): column blocks jb in order, each with the row blocks
-// ib = 0..jb on or above the diagonal.
-__device__ __forceinline__ void tile_coords(int t, int n_ib, int n_jb, int& ib, int& jb) {
-  for (jb = 0; jb < n_jb; ++jb) {
-    int cnt = min(jb + 1, n_ib);
-    if (t < cnt) { ib = t; return; }
-    t -= cnt;
-  }
-  ib = 0;  // unreachable for t < n_tiles
-}
 
 __global__ void __launch_bounds__(THREADS, 1)
 syrk_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_x,
@@ -75,6 +70,7 @@ syrk_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_x,
   uint64_t* empty = bars + STAGES;       // [STAGES]
   uint64_t* acc_full = bars + 2 * STAGES;       // accumulator complete
   uint64_t* acc_empty = bars + 2 * STAGES + 1;  // accumulator drained
+  uint64_t* mma_drain = bars + 2 * STAGES + 2;  // abort path: the issued MMAs have completed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* skip_flag = abort_flag + 1;
@@ -90,6 +86,7 @@ syrk_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_x,
     }
     gptq::mbar_init(acc_full, 1);
     gptq::mbar_init(acc_empty, EPI_WARPS);
+    gptq::mbar_init(mma_drain, 1);
     gptq::fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
@@ -112,10 +109,10 @@ syrk_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_x,
       if (lane == 0) {
         int stage = 0;
         uint32_t phase = 0;
+        uint32_t filled = 0, fill_parity = 0;  // per stage: filled at least once, last parity
         for (long long u = blockIdx.x; u < args.n_units && !*abort_flag; u += gridDim.x) {
-          const int tile = (int)(u % args.n_tiles), split = (int)(u / args.n_tiles);
-          int ib, jb;
-          tile_coords(tile, args.n_ib, args.n_jb, ib, jb);
+          int ib, jb, split;
+          gptq::syrk_unit_coords(u, args.n_tb, args.grp, args.n_split, ib, jb, split);
           const int kb0 = split * args.kb_per_split;
           const int kb1 = min(args.nkb_total, kb0 + args.kb_per_split);
           for (int kb = kb0; kb < kb1; ++kb) {
@@ -130,9 +127,14 @@ syrk_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_x,
 #pragma unroll
             for (int q = 0; q < 4; ++q)
               gptq::tma_load_2d(sb + q * BOX_BYTES, &tmap_x, &full[stage], jb * BN + q * BOX, t);
+            filled |= 1u << stage;
+            fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
             if (++stage == STAGES) { stage = 0; phase ^= 1; }
           }
         }
+        if (*abort_flag)  // let the loads already issued land before the CTA exits
+          for (int s = 0; s < STAGES; ++s)
+            if (filled & (1u << s)) gptq::mbar_drain(&full[s], (fill_parity >> s) & 1u);
       }
     } else if (warp == 1) {
       // ------------------------------- MMA issuer ---------------------------------
@@ -141,7 +143,8 @@ syrk_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_x,
         uint32_t phase = 0;
         uint32_t acc_phase = 0;
         for (long long u = blockIdx.x; u < args.n_units && !*abort_flag; u += gridDim.x) {
-          const int split = (int)(u / args.n_tiles);
+          int ib_, jb_, split;
+          gptq::syrk_unit_coords(u, args.n_tb, args.grp, args.n_split, ib_, jb_, split);
           const int kb0 = split * args.kb_per_split;
           const int kb1 = min(args.nkb_total, kb0 + args.kb_per_split);
           if (!gptq::mbar_wait(acc_empty, acc_phase ^ 1, abort_flag)) break;
@@ -174,6 +177,10 @@ syrk_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_x,
           gptq::mma_commit(acc_full);
           acc_phase ^= 1;
         }
+        if (*abort_flag) {  // the MMAs already issued finish before TMEM is released
+          gptq::mma_commit(mma_drain);
+          gptq::mbar_drain(mma_drain, 0);
+        }
       }
     } else {
       // ------------------------------- epilogue -----------------------------------
@@ -182,9 +189,8 @@ syrk_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_x,
       uint32_t acc_phase = 0;
       uint32_t chunk_counter = 0;
       for (long long u = blockIdx.x; u < args.n_units && !*abort_flag; u += gridDim.x) {
-        const int tile = (int)(u % args.n_tiles);
-        int ib, jb;
-        tile_coords(tile, args.n_ib, args.n_jb, ib, jb);
+        int ib, jb, split;
+        gptq::syrk_unit_coords(u, args.n_tb, args.grp, args.n_split, ib, jb, split);
         if (!gptq::mbar_wait(acc_full, acc_phase, abort_flag)) break;
         gptq::tc_fence_after();
 #pragma unroll 1
@@ -244,12 +250,17 @@ syrk_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_x,
   if (threadIdx.x == 0 && *abort_flag) gptq::set_status(args.status, GPTQ_ERR_TIMEOUT, 1);
 }
 
-__global__ void zero_upper_kernel(float* H, int d, long long ldh) {
-  const long long total = (long long)d * d;
-  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
-       e += (long long)gridDim.x * blockDim.x) {
-    const int i = (int)(e / d), j = (int)(e % d);
-    if (i <= j) H[i * ldh + j] = 0.0f;
+// H's upper triangle (with the diagonal) = 0 before a non-accumulating product: rows on grid y,
+// columns of the row's span strided over grid x (tri_fill.cuh), no per-element division.
+__global__ void zero_upper_kernel(float* H, int d, long long ldh, const int32_t* status) {
+  if (gptq::status_bad(status)) return;
+  for (long long r = blockIdx.y; r < d; r += gridDim.y) {
+    long long lo, hi;
+    gptq::tri_row_span(gptq::kUpperWithDiag, r, d, lo, hi);
+    float* row = H + r * ldh;
+    for (long long c = lo + blockIdx.x * (long long)blockDim.x + threadIdx.x; c < hi;
+         c += (long long)gridDim.x * blockDim.x)
+      row[c] = 0.f;
   }
 }
 
@@ -261,7 +272,8 @@ int syrk_bf16_upper(float* H, int d, long long ldh, const void* X, long long n_t
                     long long ldx, float alpha, int accumulate, int32_t* status,
                     cudaStream_t stream) {
   if (!accumulate) {
-    zero_upper_kernel<<<num_sms() * 4, 256, 0, stream>>>(H, d, ldh);
+    const dim3 grid((unsigned)((d + 1023) / 1024), (unsigned)(d < 65535 ? d : 65535));
+    zero_upper_kernel<<<grid, 256, 0, stream>>>(H, d, ldh, status);
     if (cudaGetLastError() != cudaSuccess) return GPTQ_ERR_CUDA;
   }
   if (n_tokens == 0) return GPTQ_OK;
@@ -276,10 +288,9 @@ int syrk_bf16_upper(float* H, int d, long long ldh, const void* X, long long n_t
 
   SyrkArgs a;
   a.d = d;
-  a.n_ib = (d + BM - 1) / BM;
-  a.n_jb = (d + BN - 1) / BN;
-  a.n_tiles = 0;
-  for (int jb = 0; jb < a.n_jb; ++jb) a.n_tiles += (jb + 1 < a.n_ib) ? jb + 1 : a.n_ib;
+  static_assert(BM == BN, "square tiles: one tile grid for rows and columns");
+  a.n_tb = (d + BM - 1) / BM;
+  a.n_tiles = a.n_tb * (a.n_tb + 1) / 2;
   a.nkb_total = (int)((n_tokens + BK - 1) / BK);
   // The tensor core rounds toward zero when it adds into its fp32 accumulator (a one-sided
   // error of up to one ulp per step on these like-signed sums), so one accumulator covers at
@@ -307,10 +318,20 @@ int syrk_bf16_upper(float* H, int d, long long ldh, const void* X, long long n_t
   a.n_units = (long long)a.n_tiles * a.n_split;
   a.alpha = alpha;
   a.status = status;
+  const int grid = (int)(a.n_units < sms ? a.n_units : sms);
+  // Groups: when every 256-channel panel of one token range fits in half of L2, one group (the
+  // CTAs share the whole range); otherwise grp x grp tiles with grp^2 about one wave, so the
+  // CTAs running together need 2 grp panels.
+  const double panel_bytes = (double)BM * a.kb_per_split * BK * 2.0;
+  if (a.n_tb * panel_bytes <= 64.0 * 1024 * 1024) {
+    a.grp = a.n_tb;
+  } else {
+    a.grp = (int)floor(sqrt((double)grid));
+    if (a.grp < 1) a.grp = 1;
+  }
 
   if (ensure_smem_attr(reinterpret_cast<const void*>(syrk_bf16_tcgen05_kernel), SMEM_BYTES) != 0)
     return GPTQ_ERR_CUDA;
-  const int grid = (int)(a.n_units < sms ? a.n_units : sms);
   syrk_bf16_tcgen05_kernel<<<grid, THREADS, SMEM_BYTES, stream>>>(tx, th, a);
   return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ERR_CUDA;
 }

@@ -29,8 +29,8 @@ int main(void) {
   const size_t ws = gptq_workspace_size(4096, 4096, &p);
   check(ws == (size_t)2 * 4096 * 4096 * 4, "workspace of a natural-order 4096 x 4096 layer");
   p.order = GPTQ_ORDER_DESC_ACT;
-  check(gptq_workspace_size(4096, 4096, &p) == ws + (size_t)4096 * 4096,
-        "act-order adds the sweep-order codes");
+  check(gptq_workspace_size(4096, 4096, &p) == ws + (size_t)4096 * 4096 + (size_t)4096 * 4,
+        "act-order adds the sweep-order codes and the inverse permutation");
   p.order = GPTQ_ORDER_NATURAL;
   p.bits = 5;
   check(gptq_workspace_size(4096, 4096, &p) == 0, "5-bit codes are rejected");
@@ -60,6 +60,13 @@ int main(void) {
   check(gptq_dequant_gemv(fake_q, 64, 128, 4, fake_h, fake_h, 1, -1, NULL, fake_h, 9, 128,
                           fake_f, 64, NULL) == GPTQ_ERR_INVALID_ARG,
         "gemv: batch above 8");
+
+  check(gptq_gemm_f32(8, 8, 8, 1.0f, fake_f, 8, 0, fake_f, 8, 0, 0.0f, NULL, 8, NULL, NULL) ==
+            GPTQ_ERR_INVALID_ARG,
+        "gemm: null C");
+  check(gptq_gemm_f32(8, 8, 8, 1.0f, fake_f, 4, 0, fake_f, 8, 0, 0.0f, fake_f, 8, NULL, NULL) ==
+            GPTQ_ERR_INVALID_ARG,
+        "gemm: lda shorter than a row of A");
 
   if (failures == 0) printf("ok\n");
   return failures == 0 ? 0 : 1;

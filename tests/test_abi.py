@@ -25,7 +25,8 @@ def declared_functions():
 
 def test_header_declares_the_boundary():
     assert declared_functions() == sorted([
-        "gptq_dequant_gemv", "gptq_hessian_accumulate", "gptq_pack", "gptq_prepare_hinv",
+        "gptq_dequant_gemv", "gptq_gemm_f32", "gptq_hessian_accumulate", "gptq_pack",
+        "gptq_prepare_hinv", "gptq_quantize_pack_layer",
         "gptq_quantize_layer", "gptq_quantize_layer_noalloc", "gptq_status_string",
         "gptq_workspace_size", "rtn_quantize"])
 
@@ -61,8 +62,10 @@ def test_workspace_size(lib):
     ok = P(4, 128, 0, 0, 128, 0.01)
     assert lib.gptq_workspace_size(4096, 4096, ctypes.byref(ok)) == 2 * 4096 * 4096 * 4
     act = P(3, 128, 0, 1, 128, 0.01)
-    assert lib.gptq_workspace_size(4096, 4096, ctypes.byref(act)) == 2 * 4096 * 4096 * 4 + 4096 * 4096
-    # static groups add the inverse column permutation (int32 per column)
+    # a permuted order adds the sweep-order codes and the inverse permutation (int32 per column)
+    assert lib.gptq_workspace_size(4096, 4096, ctypes.byref(act)) == \
+        2 * 4096 * 4096 * 4 + 4096 * 4096 + 4096 * 4
+    # static groups use the same inverse permutation
     st = P(4, 128, 0, 1, 128, 0.01, 1)
     assert lib.gptq_workspace_size(4096, 4096, ctypes.byref(st)) == \
         2 * 4096 * 4096 * 4 + 4096 * 4096 + 4096 * 4
@@ -130,3 +133,23 @@ def test_dequant_gemv_rejects_bad_arguments_on_host(lib):
     assert call(g=48) == 1                  # group size does not divide d_in
     assert call(G=2) == 1                   # n_groups disagrees with group_size
     assert call(g=-1, G=2) == 1
+
+
+def test_gemm_host_checks(lib):
+    """gptq_gemm_f32 rejects null pointers, impossible shapes and short leading dimensions on
+    the host (nothing is launched; the fake pointers are never dereferenced)."""
+    V, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    lib.gptq_gemm_f32.argtypes = [I64, I64, I64, ctypes.c_float, V, I64, I, V, I64, I,
+                                  ctypes.c_float, V, I64, V, V]
+    lib.gptq_gemm_f32.restype = I
+    f = 0x1000
+
+    def call(M=8, N=8, K=8, A=f, lda=8, ta=0, B=f, ldb=8, tb=0, C=f, ldc=8):
+        return lib.gptq_gemm_f32(M, N, K, 1.0, A, lda, ta, B, ldb, tb, 0.0, C, ldc, None, None)
+    assert call(C=None) == 1
+    assert call(A=None) == 1 and call(B=None) == 1
+    assert call(M=0) == 1 and call(N=0) == 1 and call(K=-1) == 1
+    assert call(lda=7) == 1 and call(ldb=7) == 1 and call(ldc=7) == 1
+    assert call(ta=1, lda=7, M=8, K=9) == 1          # op(A)^T rows are M long
+    assert call(ta=2) == 1 and call(tb=2) == 1
+    assert call(C=0x1002) == 1                        # misaligned fp32 pointer

@@ -163,3 +163,42 @@ def test_unpermute_codes_index_math_on_cpu(tmp_path, n, d):
     want = np.empty_like(cs)
     want[:, perm] = cs
     np.testing.assert_array_equal(got, want)
+
+
+@pytest.mark.skipif(shutil.which("nvcc") is None, reason="needs nvcc")
+def test_wait_timeout_check_kernel_builds(tmp_path):
+    """The test-only bounded-wait kernel (run by tests/test_gpu_failure.py) cross-compiles for
+    sm_100a against the library's own wait helpers."""
+    so = tmp_path / "wait_timeout_check.so"
+    r = subprocess.run(["nvcc", "-gencode", "arch=compute_100a,code=sm_100a", "-O2", "-shared",
+                        "-Xcompiler", "-fPIC", "-I",
+                        os.path.join(ROOT, "post_weight_quantization_18_b200", "csrc"),
+                        os.path.join(ROOT, "tests", "c", "wait_timeout_check.cu"), "-o", str(so),
+                        "-lcuda"], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+
+
+@pytest.mark.skipif(shutil.which("g++") is None, reason="needs g++")
+@pytest.mark.parametrize("n_tb,grp,n_split", [(1, 1, 1), (16, 16, 32), (16, 12, 3), (112, 12, 16),
+                                              (7, 3, 2), (5, 8, 1)])
+def test_syrk_unit_order_on_cpu(tmp_path, n_tb, grp, n_split):
+    """The SYRK's work units (syrk_units.cuh, the kernel's own mapping) cover every upper tile
+    (ib <= jb) in every token range exactly once, and inside a group run range by range."""
+    import numpy as np
+    exe = tmp_path / "syrk_units_check"
+    r = subprocess.run(["g++", "-std=c++17", "-O2", "-Wall", "-Werror",
+                        "-I", os.path.join(ROOT, "post_weight_quantization_18_b200", "csrc"),
+                        os.path.join(ROOT, "tests", "c", "syrk_units_check.cpp"), "-o", str(exe)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe), str(n_tb), str(grp), str(n_split)], capture_output=True,
+                       text=True, timeout=120)
+    assert r.returncode == 0, r.stderr
+    got = np.array([list(map(int, line.split())) for line in r.stdout.splitlines()])
+    want = {(i, j, s) for j in range(n_tb) for i in range(j + 1) for s in range(n_split)}
+    assert len(got) == len(want) and {tuple(x) for x in got} == want
+    # consecutive units of one group share the token range until the group's tiles are done
+    grp_id = (got[:, 0] // grp) * 100000 + (got[:, 1] // grp)
+    for g in np.unique(grp_id):
+        splits = got[grp_id == g, 2]
+        assert np.all(np.diff(splits) >= 0)

@@ -86,3 +86,22 @@ def test_graph_replay_matches_direct_calls(n, d, N, bits, g, sym, order):
         rel = np.linalg.norm(h_rep - h_dir) / np.linalg.norm(h_dir)
         assert rel <= 1e-6, rel
     del graph
+
+
+def test_bench_counts_kernel_launches_from_recorded_graphs():
+    """bench.py reports the kernels a step launches as the kernel nodes of the CUDA graphs it
+    records from the C ABI calls; the count is positive and the same for two recordings."""
+    import bench
+    import post_weight_quantization_18_b200 as G
+    from gpu_util import make_inputs
+    W, X = make_inputs(64, 512, 4096, seed=5)
+    Wd, Xd = W.cuda(), X.cuda()
+    G.quantize_layer(Wd, X=Xd)              # first call: stream and attribute set-up
+    torch.cuda.synchronize()
+    counts = []
+    for _ in range(2):
+        gr, kept = bench.new_graph()
+        with torch.cuda.graph(gr):
+            G.quantize_layer(Wd, X=Xd, check=False)
+        counts.append(bench.graph_kernel_nodes(gr) if kept else None)
+    assert counts[0] is not None and counts[0] > 5 and counts[0] == counts[1], counts

@@ -33,8 +33,7 @@ def test_act_order_given_perm_matches_oracle():
 
 def test_act_order_desc_act_on_gpu():
     W, X = make_inputs(128, 384, 5000, seed=78)
-    compare_with_oracle(W, X, bits=4, group_size=128, act_order=True, given_perm=False,
-                        code_agree=0.99, err_rtol=5e-3)
+    compare_with_oracle(W, X, bits=4, group_size=128, act_order=True, given_perm=False)
 
 
 def test_fp32_small_workload():
@@ -119,8 +118,7 @@ def test_static_groups_act_order_given_perm_matches_oracle():
 
 def test_static_groups_desc_act_on_gpu():
     W, X = make_inputs(160, 384, 5000, seed=92, half_normal=True)
-    compare_with_oracle(W, X, bits=3, group_size=128, act_order=True, static_groups=True,
-                        err_rtol=5e-3)
+    compare_with_oracle(W, X, bits=3, group_size=128, act_order=True, static_groups=True)
 
 
 def test_static_groups_natural_order_g64_sym():

@@ -50,10 +50,3 @@ def test_two_gloo_ranks_max_and_disjoint_seeds():
 def test_single_process_identity():
     import bench
     assert bench.max_over_ranks([1.5, 2.5], "cpu") == [1.5, 2.5]
-
-
-def test_launch_accounting_matches_recursions():
-    """The bench's launch count follows the host recursions (d = 4096: 288 per step)."""
-    import bench
-    import layer_inputs as li
-    assert bench.launches_per_step(4096, li.WORKLOADS["llama7b_attn_proj"].quant) == 288
