@@ -379,7 +379,7 @@ SweepStreams* sweep_streams() {
   return &ss;
 }
 
-constexpr int kPanelMinRows = 1024;  // below this one panel (the leaves do not fill the GPU)
+constexpr int kPanelMinRows = 8192;  // below this one panel: half the rows make the products too small
 
 int sweep_in_panels(const SweepCtx& c) {
   const int n1 = ((c.n / 2 + 15) / 16) * 16;  // whole 16-row sweep CTAs in the first panel

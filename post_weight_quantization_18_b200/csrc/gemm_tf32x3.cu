@@ -15,8 +15,9 @@
 //               both into tensor memory (tcgen05.st); together they write the lo part of the B
 //               tile to a second buffer (the landed tile itself is B's hi operand: the tensor core
 //               reads an fp32 operand of kind::tf32 as its top 19 bits)
-//   warps 6-9   epilogue: each thread owns one row of the tile and adds the accumulator of every
-//               K stretch into registers (fp32, round to nearest), then writes C once
+//   warps 6-13  epilogue: two warps per TMEM lane quarter; each thread owns half a row of the
+//               tile (64 columns) and adds the accumulator of every K stretch into registers
+//               (fp32, round to nearest), then writes C once
 // Shared memory is the limiting resource of the three-product scheme: with A in tensor memory the
 // MMAs read only B from it, about half of what reading both operands three times would take.
 //
@@ -39,8 +40,9 @@ constexpr int TILE_BYTES = 128 * BK * 4;              // 16 KB: one operand tile
 constexpr int STAGE_BYTES = 3 * TILE_BYTES;           // A (for the converters), B, B_lo
 constexpr int SMEM_DATA = STAGES * STAGE_BYTES;       // 192 KB
 constexpr int SMEM_BYTES = SMEM_DATA + 1024 + 256;
-constexpr int THREADS = 320;
-constexpr int CONV_WARP0 = 2, N_CONV = 4, EPI_WARP0 = 6, N_EPI = 4;
+constexpr int THREADS = 448;
+constexpr int CONV_WARP0 = 2, N_CONV = 4, EPI_WARP0 = 6, N_EPI = 8;
+constexpr int EPI_COLS = BN / 2;     // columns of a row per epilogue thread (two warps per quarter)
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;      // two 128-column accumulators, at columns 0 and 128
 constexpr uint32_t A_COL = 256;      // stage s: A_hi at A_COL + 64 s, A_lo at A_COL + 64 s + 32
@@ -298,6 +300,7 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
     } else {
       // ---------------- epilogue: K stretches summed in registers ----------------
       const int quarter = warp & 3;
+      const int col_half = (warp - EPI_WARP0) >> 2;  // columns [64 col_half, 64 col_half + 64)
       const uint32_t lane_field = (uint32_t)(quarter * 32) << 16;
       int buf = 0;
       uint32_t acc_phase = 0;
@@ -307,23 +310,24 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
         if (!tile_live(tm, tn, args)) continue;
         int kb0, kb1;
         tile_kb(tm, tn, args, nkb, kb0, kb1);
-        float acc[BN];
+        float acc[EPI_COLS];
 #pragma unroll
-        for (int e = 0; e < BN; ++e) acc[e] = 0.f;  // 0 + x is x exactly: no select per element
+        for (int e = 0; e < EPI_COLS; ++e) acc[e] = 0.f;  // 0 + x is x exactly: no select
         bool ok = true;
         for (int kc = kb0; kc < kb1; kc += KCB) {
           if (!gptq::mbar_wait(&acc_full[buf], acc_phase, abort_flag)) { ok = false; break; }
           gptq::tc_fence_after();
 #pragma unroll
-          for (int q = 0; q < BN / 16; ++q) {  // 16 columns per load: acc[] stays in registers
-            uint32_t r[16];
+          for (int q = 0; q < EPI_COLS / 32; ++q) {
+            uint32_t r[32];
             __syncwarp();  // tcgen05.ld is warp-collective: reconverge before every load
-            gptq::tmem_ld_32x32b_x16(tmem_base + lane_field + ACC_COL + (uint32_t)(buf * BN + 16 * q),
+            gptq::tmem_ld_32x32b_x32(tmem_base + lane_field + ACC_COL +
+                                         (uint32_t)(buf * BN + EPI_COLS * col_half + 32 * q),
                                      r);
             gptq::tmem_ld_wait();
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
-              acc[16 * q + e] += __uint_as_float(r[e]);
+            for (int e = 0; e < 32; ++e)
+              acc[32 * q + e] += __uint_as_float(r[e]);
           }
           gptq::tc_fence_before();
           __syncwarp();
@@ -336,8 +340,8 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
           float* crow = args.C + (long long)row * args.ldc;
           const float alpha = args.alpha, beta = args.beta;
 #pragma unroll
-          for (int c = 0; c < BN / 32; ++c) {
-            const int col0 = tn * BN + c * 32;
+          for (int c = 0; c < EPI_COLS / 32; ++c) {
+            const int col0 = tn * BN + EPI_COLS * col_half + c * 32;
             if (col0 >= args.N) continue;
             const bool full_vec = (col0 + 32 <= args.N) && (!args.upper_only || row <= col0);
             if (full_vec) {

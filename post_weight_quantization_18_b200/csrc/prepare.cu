@@ -123,16 +123,14 @@ __global__ void dead_damp_kernel(float* __restrict__ H, uint8_t* __restrict__ de
   for (int j = threadIdx.x; j < d; j += blockDim.x) H[(long long)j * d + j] += lam;
 }
 
-// U's strictly lower triangle = 0: rows on grid y, columns strided over grid x (tri_fill.cuh).
+// U's strictly lower triangle = 0: rows over the blocks, 16-byte stores along each row's span
+// (tri_fill.cuh).
 __global__ void zero_lower_kernel(float* U, int d, const int32_t* status) {
   if (gptq::status_bad(status)) return;
-  for (long long r = blockIdx.y; r < d; r += gridDim.y) {
+  for (long long r = blockIdx.x; r < d; r += gridDim.x) {
     long long lo, hi;
     gptq::tri_row_span(gptq::kStrictLower, r, d, lo, hi);
-    float* row = U + r * d;
-    for (long long c = lo + blockIdx.x * (long long)blockDim.x + threadIdx.x; c < hi;
-         c += (long long)gridDim.x * blockDim.x)
-      row[c] = 0.f;
+    gptq::fill_span(U + r * d, lo, hi, 0.f, threadIdx.x, blockDim.x);
   }
 }
 
@@ -453,7 +451,7 @@ int prep_dead_damp(float* H, uint8_t* dead, int d, float percdamp, int32_t* stat
 }
 
 int prep_zero_lower(float* U, int d, const int32_t* status, cudaStream_t stream) {
-  const dim3 grid((unsigned)((d + 1023) / 1024), (unsigned)(d < 65535 ? d : 65535));
+  const int grid = d < num_sms() * 8 ? d : num_sms() * 8;
   zero_lower_kernel<<<grid, 256, 0, stream>>>(U, d, status);
   return cudaGetLastError() == cudaSuccess ? 0 : GPTQ_ERR_CUDA;
 }

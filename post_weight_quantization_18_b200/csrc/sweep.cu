@@ -15,11 +15,12 @@
 // Layout: eight lanes own one row (four rows per warp); in each 32-column chunk of the block,
 // lane s of a row holds the four contiguous columns 4s..4s+3, so one row of U is read with
 // float4 loads, the remaining columns are spread evenly over the lanes, and chunks that are
-// already quantized are skipped uniformly. For column j the owner lane's value is broadcast
-// inside its 8-lane group, the group evaluates the quantizer, and the owner keeps the code and
-// the error in registers; when a chunk is done every lane stores its four codes (one 32-bit
-// word) and errors (one float4). The block's U (128 x 128, zero below the diagonal as gptq_prepare_hinv writes it)
-// arrives in shared memory with one TMA copy; 1/U_jj is computed from it.
+// already quantized are skipped uniformly. For column j the owner lane evaluates the quantizer
+// on its own value and broadcasts the error inside its 8-lane group; it keeps the code and the
+// error in registers, and when a chunk is done every lane stores its four codes (one 32-bit
+// word) and errors (one float4). The block's U (128 x 128, zero below the diagonal as
+// gptq_prepare_hinv writes it) arrives in shared memory with one TMA copy; 1/U_jj is computed
+// from it.
 #include <float.h>
 
 #include <cuda_bf16.h>
@@ -47,10 +48,12 @@ constexpr int SW_SMEM_STATIC = SW_SMEM + 3 * 16 * BLK * 4 + BLK * 4;  // + (s, 1
 // rint(t) equals rint(w / s) unless t lies within that distance of a rounding boundary
 // (k + 1/2); only then is the quotient formed exactly. The margin used, 2^-21 |t|, covers the
 // bound with room to spare.
-__device__ __forceinline__ float quant_code_rcp(float w, float s, float rs, float z, float maxq) {
+// Lanes whose result is not used (exact = false) skip the exact quotient.
+__device__ __forceinline__ float quant_code_rcp(float w, float s, float rs, float z, float maxq,
+                                                bool exact = true) {
   float t = w * rs;
   float r = rintf(t);
-  if (fabsf(fabsf(t - r) - 0.5f) <= 4.76837158e-7f * fabsf(t)) r = rintf(__fdiv_rn(w, s));
+  if (exact && fabsf(fabsf(t - r) - 0.5f) <= 4.76837158e-7f * fabsf(t)) r = rintf(__fdiv_rn(w, s));
   return fminf(fmaxf(r + z, 0.0f), maxq);
 }
 
@@ -76,6 +79,44 @@ __device__ __forceinline__ float group8_max(float v) {
   v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
   v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
   return fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+}
+
+// (s, z, 1/s) of the group that starts at block column j, from the current values of its g
+// columns (min / max over the row's eight lanes; w[4c + e] holds column 32c + 4 sub + e), and the
+// stores of (s, z) (and their fp16 copies for the packed output) by the row's first lane.
+__device__ __forceinline__ float3 group_params(const float (&w)[16], int j, int g, int sub,
+                                               bool sym, int bits, float maxq, bool store,
+                                               long long gi, float* scales, float* zeros,
+                                               uint16_t* s16, uint16_t* z16) {
+  float a = sym ? 0.f : FLT_MAX, b = -FLT_MAX, s, z;
+#pragma unroll
+  for (int c2 = 0; c2 < 4; ++c2)
+#pragma unroll
+    for (int e2 = 0; e2 < 4; ++e2) {
+      const int k = 32 * c2 + 4 * sub + e2;
+      const float v = w[4 * c2 + e2];
+      if (k >= j && k < j + g) {
+        if (sym) a = fmaxf(a, fabsf(v));
+        else { a = fminf(a, v); b = fmaxf(b, v); }
+      }
+    }
+  if (sym) {
+    a = group8_max(a);
+    sym_params(a, bits, s, z);
+  } else {
+    a = group8_min(a);
+    b = group8_max(b);
+    asym_params(a, b, maxq, s, z);
+  }
+  if (store) {
+    scales[gi] = s;
+    zeros[gi] = z;
+    if (s16 != nullptr) {  // packed output: the fp16 copies (round to nearest even)
+      s16[gi] = __half_as_ushort(__float2half_rn(s));
+      z16[gi] = __half_as_ushort(__float2half_rn(z));
+    }
+  }
+  return make_float3(s, z, __frcp_rn(s));
 }
 
 // 32 codes (c[i]: codes 4i .. 4i+3 as bytes) -> `bits` words of the packed row at out, the
@@ -106,7 +147,7 @@ __device__ __forceinline__ void store_packed_chunk(const uint32_t (&c)[8], int b
 // STATIC: static groups (one instance each, so the default path carries no extra branch).
 // FINE: groups shorter than 32 columns, whose starts fall inside a 32-column chunk.
 template <bool STATIC, bool FINE>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(128, 4)
 sweep_block_kernel(const __grid_constant__ CUtensorMap tmap_u, const float* __restrict__ Wwork,
                    float* __restrict__ Err, uint8_t* __restrict__ codes,
                    float* __restrict__ scales, float* __restrict__ zeros, int n, int d, int col0,
@@ -190,75 +231,94 @@ sweep_block_kernel(const __grid_constant__ CUtensorMap tmap_u, const float* __re
   uint8_t* crow = codes + (long long)rsafe * d + col0;
   const bool codes_vec = (reinterpret_cast<uintptr_t>(codes) & 3) == 0 && (d & 3) == 0;
   bool finite = true;
-  // (s, z) of the group that starts at block column j, from the current values of its g
-  // columns (min / max over the row's eight lanes).
-  auto group_params = [&](int j) {
-    float a = sym ? 0.f : FLT_MAX, b = -FLT_MAX;
-#pragma unroll
-    for (int c2 = 0; c2 < 4; ++c2)
-#pragma unroll
-      for (int e2 = 0; e2 < 4; ++e2) {
-        const int k = 32 * c2 + 4 * sub + e2;
-        const float v = w[4 * c2 + e2];
-        if (k >= j && k < j + g) {
-          if (sym) a = fmaxf(a, fabsf(v));
-          else { a = fminf(a, v); b = fmaxf(b, v); }
-        }
-      }
-    if (sym) {
-      a = group8_max(a);
-      sym_params(a, bits, s, z);
-    } else {
-      a = group8_min(a);
-      b = group8_max(b);
-      asym_params(a, b, maxq, s, z);
-    }
-    rs = __frcp_rn(s);
-    if (sub == 0 && live) {
-      const long long gi = (long long)row * G + (col0 + j) / g;
-      scales[gi] = s;
-      zeros[gi] = z;
-      if (s16 != nullptr) {  // packed output: the fp16 copies (round to nearest even)
-        s16[gi] = __half_as_ushort(__float2half_rn(s));
-        z16[gi] = __half_as_ushort(__float2half_rn(z));
-      }
-    }
-  };
 #pragma unroll
   for (int c = 0; c < 4; ++c) {                  // 32-column chunks
     float qk[4], ek[4];                          // this lane's four codes and errors of chunk c
     // Groups of 32 columns or more start at chunk starts: their statistics are taken here,
     // outside the column loop (which keeps that loop's unrolled code small).
-    if (!FINE && grouped && ((32 * c) & gmask) == 0) group_params(32 * c);
+    if (!FINE && grouped && ((32 * c) & gmask) == 0) {
+      const float3 p = group_params(w, 32 * c, g, sub, sym, bits, maxq, sub == 0 && live,
+                                    (long long)row * G + (col0 + 32 * c) / g, scales, zeros,
+                                    s16, z16);
+      s = p.x; z = p.y; rs = p.z;
+    }
+    // Columns 32c + 4 so + e: lane so of the row's group owns the four of a run. Every lane
+    // quantizes its own slot (only the owner's result is kept), so the owner needs no broadcast
+    // to decide a column; the error is then broadcast for the other lanes' updates. The owner
+    // forms its next column's value from its own error, and that next decision is written
+    // before this column's updates, which wait on the broadcast: issue is in order, so the
+    // decisions of a run follow one another without the broadcast in between. Only the step to
+    // the next lane's run waits on it. (Groups shorter than 32 columns take their statistics
+    // inside the run from every lane's updated values, so that case keeps the plain order.)
 #pragma unroll 1
     for (int so = 0; so < 8; ++so) {             // owner sub-lane within the chunk
+      const bool owner = sub == so;
+      const int j0 = 32 * c + 4 * so;
+      if (STATIC) {
+        s = stab[rl * BLK + j0];
+        rs = stab[16 * BLK + rl * BLK + j0];
+        z = stab[32 * BLK + rl * BLK + j0];
+      } else if (FINE && (j0 & gmask) == 0) {
+        const float3 p = group_params(w, j0, g, sub, sym, bits, maxq, sub == 0 && live,
+                                      (long long)row * G + (col0 + j0) / g, scales, zeros, s16,
+                                      z16);
+        s = p.x; z = p.y; rs = p.z;
+      }
+      float xcur = w[4 * c];                     // the owner's column j0, up to date
+      float qv = quant_code_rcp(xcur, s, rs, z, maxq, owner);
+      float eo = (xcur - s * (qv - z)) * invd[j0];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int j = 32 * c + 4 * so + e;
-        if (STATIC) {
-          s = stab[rl * BLK + j];
-          rs = stab[16 * BLK + rl * BLK + j];
-          z = stab[32 * BLK + rl * BLK + j];
-        } else if (FINE && (j & gmask) == 0) {
-          group_params(j);
-        }
-        const float wj = __shfl_sync(0xffffffffu, w[4 * c + e], grp | so);
-        const float qv = quant_code_rcp(wj, s, rs, z, maxq);
-        const float err = (wj - s * (qv - z)) * invd[j];
-        if (sub == so) {
+        const int j = j0 + e;
+        const float err = __shfl_sync(0xffffffffu, eo, grp | so);
+        if (owner) {
           qk[e] = qv;
-          ek[e] = err;
+          ek[e] = eo;
         }
         finite = finite && (fabsf(err) <= FLT_MAX);
-        // w_k -= err * U_jk for the columns of chunks c..3 (U_jk = 0 for k < j).
         const float* urow = Us + j * BLK + 4 * sub;
+        const float4 uc = *reinterpret_cast<const float4*>(urow + 32 * c);
+        float qn = 0.f, en = 0.f;
+        if (!FINE && e < 3) {
+          // column j + 1: the owner's value from its own error, decided before the updates
+          const float un = e == 0 ? uc.y : (e == 1 ? uc.z : uc.w);
+          const float xn = fmaf(-eo, un, w[4 * c + e + 1]);
+          if (STATIC) {
+            s = stab[rl * BLK + j + 1];
+            rs = stab[16 * BLK + rl * BLK + j + 1];
+            z = stab[32 * BLK + rl * BLK + j + 1];
+          }
+          qn = quant_code_rcp(xn, s, rs, z, maxq, owner);
+          en = (xn - s * (qn - z)) * invd[j + 1];
+        }
+        // w_k -= err * U_jk for the columns of chunks c..3 (U_jk = 0 for k < j).
+        w[4 * c + 0] = fmaf(-err, uc.x, w[4 * c + 0]);
+        w[4 * c + 1] = fmaf(-err, uc.y, w[4 * c + 1]);
+        w[4 * c + 2] = fmaf(-err, uc.z, w[4 * c + 2]);
+        w[4 * c + 3] = fmaf(-err, uc.w, w[4 * c + 3]);
 #pragma unroll
-        for (int c2 = c; c2 < 4; ++c2) {
+        for (int c2 = c + 1; c2 < 4; ++c2) {
           const float4 u = *reinterpret_cast<const float4*>(urow + 32 * c2);
           w[4 * c2 + 0] = fmaf(-err, u.x, w[4 * c2 + 0]);
           w[4 * c2 + 1] = fmaf(-err, u.y, w[4 * c2 + 1]);
           w[4 * c2 + 2] = fmaf(-err, u.z, w[4 * c2 + 2]);
           w[4 * c2 + 3] = fmaf(-err, u.w, w[4 * c2 + 3]);
+        }
+        if (e < 3) {
+          if (FINE) {  // plain order: statistics (at a group start) and decision after updates
+            const int jn = j + 1;
+            if ((jn & gmask) == 0) {
+              const float3 p = group_params(w, jn, g, sub, sym, bits, maxq, sub == 0 && live,
+                                            (long long)row * G + (col0 + jn) / g, scales, zeros,
+                                            s16, z16);
+              s = p.x; z = p.y; rs = p.z;
+            }
+            xcur = w[4 * c + e + 1];
+            qn = quant_code_rcp(xcur, s, rs, z, maxq, owner);
+            en = (xcur - s * (qn - z)) * invd[jn];
+          }
+          qv = qn;
+          eo = en;
         }
       }
     }

@@ -250,17 +250,14 @@ syrk_bf16_tcgen05_kernel(const __grid_constant__ CUtensorMap tmap_x,
   if (threadIdx.x == 0 && *abort_flag) gptq::set_status(args.status, GPTQ_ERR_TIMEOUT, 1);
 }
 
-// H's upper triangle (with the diagonal) = 0 before a non-accumulating product: rows on grid y,
-// columns of the row's span strided over grid x (tri_fill.cuh), no per-element division.
+// H's upper triangle (with the diagonal) = 0 before a non-accumulating product: rows over the
+// blocks, 16-byte stores along each row's span (tri_fill.cuh).
 __global__ void zero_upper_kernel(float* H, int d, long long ldh, const int32_t* status) {
   if (gptq::status_bad(status)) return;
-  for (long long r = blockIdx.y; r < d; r += gridDim.y) {
+  for (long long r = blockIdx.x; r < d; r += gridDim.x) {
     long long lo, hi;
     gptq::tri_row_span(gptq::kUpperWithDiag, r, d, lo, hi);
-    float* row = H + r * ldh;
-    for (long long c = lo + blockIdx.x * (long long)blockDim.x + threadIdx.x; c < hi;
-         c += (long long)gridDim.x * blockDim.x)
-      row[c] = 0.f;
+    gptq::fill_span(H + r * ldh, lo, hi, 0.f, threadIdx.x, blockDim.x);
   }
 }
 
@@ -272,7 +269,7 @@ int syrk_bf16_upper(float* H, int d, long long ldh, const void* X, long long n_t
                     long long ldx, float alpha, int accumulate, int32_t* status,
                     cudaStream_t stream) {
   if (!accumulate) {
-    const dim3 grid((unsigned)((d + 1023) / 1024), (unsigned)(d < 65535 ? d : 65535));
+    const int grid = d < num_sms() * 8 ? d : num_sms() * 8;
     zero_upper_kernel<<<grid, 256, 0, stream>>>(H, d, ldh, status);
     if (cudaGetLastError() != cudaSuccess) return GPTQ_ERR_CUDA;
   }

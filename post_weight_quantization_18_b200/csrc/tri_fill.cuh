@@ -1,9 +1,12 @@
-// tri_fill.cuh — which elements of a row-major square matrix a triangle-clearing launch
-// writes. Rows go to the grid's y dimension (grid-stride), and the threads of the x dimension
-// stride along the row's span. No per-element division: the row is known and the span is
-// contiguous. Host-and-device code, so that the kernels' index arithmetic is also checked on
-// the CPU.
+// tri_fill.cuh — which elements of a row-major square matrix a triangle launch touches. The
+// fills (zeroing a triangle) give each block whole rows (grid-stride over rows) and stride its
+// threads along the row's span with 16-byte stores; the element-wise copies put rows on the
+// grid's y dimension and stride the x dimension's threads along the span. No per-element
+// division: the row is known and the span is contiguous. Host-and-device code, so that the
+// kernels' index arithmetic is also checked on the CPU.
 #pragma once
+
+#include <stdint.h>
 
 #include "hd.cuh"
 
@@ -23,6 +26,25 @@ GPTQ_HD void tri_row_span(int part, long long r, int d, long long& lo, long long
     lo = 0;
     hi = d;
   }
+}
+
+// Thread t of nt writes v into elements [lo, hi) of the row at p: a scalar head up to the first
+// 16-byte boundary, 16-byte stores for the body, a scalar tail. (The host build, used by the
+// CPU checks, writes the body's four values one by one at the same indices.)
+GPTQ_HD void fill_span(float* p, long long lo, long long hi, float v, int t, int nt) {
+  const long long mis = (long long)((reinterpret_cast<uintptr_t>(p + lo) >> 2) & 3);
+  long long body0 = lo + ((4 - mis) & 3);
+  if (body0 > hi) body0 = hi;
+  for (long long c = lo + t; c < body0; c += nt) p[c] = v;
+  const long long quads = (hi - body0) / 4;
+  for (long long k = t; k < quads; k += nt) {
+#if defined(__CUDA_ARCH__)
+    reinterpret_cast<float4*>(p + body0)[k] = make_float4(v, v, v, v);
+#else
+    for (int e = 0; e < 4; ++e) p[body0 + 4 * k + e] = v;
+#endif
+  }
+  for (long long c = body0 + 4 * quads + t; c < hi; c += nt) p[c] = v;
 }
 
 // Codes back in the original column order: codes[r][perm[k]] = cs[r][k] (rows of d codes).

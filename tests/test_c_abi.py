@@ -85,12 +85,14 @@ def test_w_gather_code_on_cpu(tmp_path, dtype, n, d, ldw):
 
 
 @pytest.mark.skipif(shutil.which("g++") is None, reason="needs g++")
-@pytest.mark.parametrize("part,d,ld", [(0, 1, 1), (0, 37, 37), (0, 1500, 1500), (1, 37, 40),
-                                       (1, 1500, 1504)])
-def test_triangle_clear_index_math_on_cpu(tmp_path, part, d, ld):
-    """The triangle-clearing kernels' index arithmetic (tri_fill.cuh) over the host's launch grid
+@pytest.mark.parametrize("part,d,ld,grid", [(0, 1, 1, 1), (0, 37, 37, 37), (0, 1500, 1500, 1184),
+                                            (0, 1501, 1501, 3), (1, 37, 40, 37),
+                                            (1, 1500, 1504, 1184), (1, 999, 1003, 7)])
+def test_triangle_clear_index_math_on_cpu(tmp_path, part, d, ld, grid):
+    """The triangle-clearing kernels' index arithmetic (tri_fill.cuh: row spans, a scalar head
+    to a 16-byte boundary, 16-byte body, scalar tail) over a launch grid of whole rows per block
     clears exactly the strictly lower triangle (part 0) or the upper triangle with the diagonal
-    (part 1, padded rows left alone) and nothing else."""
+    (part 1, padded rows left alone) and nothing else, for rows of any alignment."""
     import numpy as np
     exe = tmp_path / "tri_fill_check"
     r = subprocess.run(["g++", "-std=c++17", "-O2", "-Wall", "-Werror",
@@ -98,8 +100,8 @@ def test_triangle_clear_index_math_on_cpu(tmp_path, part, d, ld):
                         os.path.join(ROOT, "tests", "c", "tri_fill_check.cpp"), "-o", str(exe)],
                        capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
-    r = subprocess.run([str(exe), str(part), str(d), str(ld)], capture_output=True, text=True,
-                       timeout=120)
+    r = subprocess.run([str(exe), str(part), str(d), str(ld), str(grid)], capture_output=True,
+                       text=True, timeout=120)
     assert r.returncode == 0, r.stderr
     got = np.array([[c == "1" for c in line] for line in r.stdout.split()], dtype=bool)
     want = np.ones((d, ld), bool)
