@@ -175,18 +175,22 @@ class ClockSampler:
 
 class OracleSample:
     """The FP64 oracle on a bounded sample of one layer of the workload. Both the cpu_baseline
-    key of our arm and the reference arm use this one definition:
-      * H over the first `tokens` calibration tokens (all d channels), scaled by N / tokens
-        (H is a sum over tokens);
-      * the prepare (act-order, dead columns, damping, U) at the full d, on that sample's H:
-        timed once per process and reused by every step (its cost does not depend on the
-        values);
-      * the blocked sweep and the pack of the first `rows` rows of W at the full d, scaled by
-        d_out / rows.
-    A step is one H sample plus one sweep-and-pack sample; the whole layer's time is
-    extrapolated from the step and the one prepare."""
+    key of our arm and the reference arm use this one definition. A step times:
+      * the oracle's H on the leading `hcols` channels of X over the first t1 and over the first
+        t2 calibration tokens. The cost of H at a fixed width is a fixed part (allocating,
+        mirroring and scaling the d x d result) plus a part linear in the tokens (the rank-k
+        update), so the two timings give the line that is extrapolated to all N tokens; both
+        parts grow with the entries of H, so the block's cost scales to the full d by
+        (d / hcols)^2;
+      * the blocked sweep and the pack at the full d of the first r1 and of the first r2 rows
+        of W, with U from the prepare below; the sweep's cost is a fixed per-column part plus a
+        part linear in the rows, so the two timings give the line that is extrapolated to all
+        d_out rows.
+    The prepare (act-order, dead columns, damping, U) runs once per process at the full d, on
+    H over the first t2 tokens (its cost does not depend on the values), and is counted once.
+    The whole layer's time is the sum of the three extrapolations."""
 
-    def __init__(self, wl, tokens, rows):
+    def __init__(self, wl, tokens=(256, 1024), rows=(16, 64), hcols=7168):
         import torch
 
         import layer_inputs as li
@@ -194,25 +198,31 @@ class OracleSample:
         lin = wl.linears[0]
         act = wl.act(lin.act)
         self.N, self.d, self.n = act.n_tokens, lin.d_in, lin.d_out
-        self.tokens, self.rows = min(tokens, act.n_tokens), min(rows, lin.d_out)
+        self.t1, self.t2 = (min(t, act.n_tokens) for t in tokens)
+        self.r1, self.r2 = (min(r, lin.d_out) for r in rows)
+        self.hcols = min(hcols, lin.d_in)
         # The first rows of the full workload's X and W (same seeded streams, same order).
-        self.X = li.activations(self.tokens, act.d, chan_sigma=act.chan_sigma,
+        self.X = li.activations(self.t2, act.d, chan_sigma=act.chan_sigma,
                                 outlier_frac=act.outlier_frac, outlier_mult=act.outlier_mult,
                                 half_normal=act.half_normal, dtype=torch.bfloat16, seed=act.seed)
-        self.W = li.weight(self.rows, lin.d_in, lin.sigma, torch.bfloat16, lin.seed)
+        self.W = li.weight(self.r2, lin.d_in, lin.sigma, torch.bfloat16, lin.seed)
         self.P = None
         self.prepare_s = None
 
-    def _hessian(self):
-        from oracle import hessian as hs
-        t0 = time.perf_counter()
-        H = hs.hessian(self.X)
-        return H, time.perf_counter() - t0
+    @staticmethod
+    def _fit(x1, y1, x2, y2, x):
+        """Value at x of the line through (x1, y1) and (x2, y2); a negative slope (timing noise)
+        counts as flat. With x1 == x2 (a workload smaller than both samples) plain scaling."""
+        if x2 == x1:
+            return y1 * x / x1
+        slope = max((y2 - y1) / (x2 - x1), 0.0)
+        return y2 + slope * (x - x2)
 
     def prepare_once(self):
+        from oracle import hessian as hs
         from oracle import prepare as prep
         q = self.wl.quant
-        H, _ = self._hessian()
+        H = hs.hessian(self.X)
         t0 = time.perf_counter()
         self.P = prep.prepare(H, self.W.double().numpy(), q.percdamp, act_order=q.act_order)
         self.prepare_s = time.perf_counter() - t0
@@ -221,30 +231,38 @@ class OracleSample:
 
     def step(self):
         """One sample step. Returns (seconds the step took, its parts)."""
+        from oracle import hessian as hs
         from oracle import pack as pk
         from oracle import sweep as sw
         q = self.wl.quant
-        t0 = time.perf_counter()
-        _, t_h = self._hessian()
-        t1 = time.perf_counter()
-        codes, S, Z, _ = sw.sweep_blocked(self.P["W"], self.P["U"], q.bits, q.group_size, q.sym,
-                                          q.block_size)
-        pk.pack(codes, S, Z, q.bits)
-        t2 = time.perf_counter()
-        return t2 - t0, dict(hessian_s=t_h, sweep_pack_s=t2 - t1)
+        parts = {}
+        t_start = time.perf_counter()
+        for key, t in (("h1", self.t1), ("h2", self.t2)):
+            t0 = time.perf_counter()
+            hs.hessian(self.X[:t, :self.hcols])
+            parts[key] = time.perf_counter() - t0
+        for key, r in (("s1", self.r1), ("s2", self.r2)):
+            t0 = time.perf_counter()
+            codes, S, Z, _ = sw.sweep_blocked(self.P["W"][:r], self.P["U"], q.bits, q.group_size,
+                                              q.sym, q.block_size)
+            pk.pack(codes, S, Z, q.bits)
+            parts[key] = time.perf_counter() - t0
+        return time.perf_counter() - t_start, parts
 
     def layer_seconds(self, parts):
-        return (parts["hessian_s"] * self.N / self.tokens + self.prepare_s +
-                parts["sweep_pack_s"] * self.n / self.rows)
+        h = self._fit(self.t1, parts["h1"], self.t2, parts["h2"], self.N)
+        h *= (self.d / self.hcols) ** 2
+        sweep = self._fit(self.r1, parts["s1"], self.r2, parts["s2"], self.n)
+        return h + self.prepare_s + sweep
 
     def describe(self):
-        return (f"FP64 oracle: H over {self.tokens} of {self.N} tokens (x{self.N / self.tokens:.0f}),"
-                f" the full {self.d}x{self.d} prepare once per process "
-                f"({self.prepare_s:.1f} s), blocked sweep and pack of {self.rows} of {self.n} rows "
-                f"(x{self.n / self.rows:.0f}); layer time extrapolated from these")
+        return (f"FP64 oracle: H on {self.hcols} of {self.d} channels over {self.t1} and "
+                f"{self.t2} of {self.N} tokens (line in the token count, x{(self.d / self.hcols) ** 2:.0f} "
+                f"for the full d x d), the full {self.d}x{self.d} prepare once per process "
+                f"({self.prepare_s:.1f} s), blocked sweep and pack of {self.r1} and {self.r2} of "
+                f"{self.n} rows at the full d (line in the row count); layer time = the sum")
 
 
-ORACLE_TOKENS, ORACLE_ROWS = 4096, 256
 
 
 def cpu_cores():
@@ -264,7 +282,7 @@ def run_reference(args):
         return
     wl = workload(args)
     lin = wl.linears[0]
-    smp = OracleSample(wl, ORACLE_TOKENS, ORACLE_ROWS)
+    smp = OracleSample(wl)
     smp.prepare_once()
     for _ in range(args.warmup):
         smp.step()
@@ -619,7 +637,7 @@ def run_ours(args):
         }
         cpu = None
         if not args.no_cpu_baseline and world == 1:
-            smp = OracleSample(wl, ORACLE_TOKENS, ORACLE_ROWS)
+            smp = OracleSample(wl)
             smp.prepare_once()
             _, parts = smp.step()
             cpu = {"value": weights / smp.layer_seconds(parts), "unit": UNIT,
