@@ -9,6 +9,7 @@
  *   gptq_quantize_pack_layer the sweep writing the packed words and fp16 scales/zeros directly
  *   rtn_quantize             round-to-nearest baseline with the same quantizer
  *   gptq_dequant_gemv        Y = X W_hat^T on the packed layer (batch 1 to 8), the format's consumer
+ *   gptq_dequant_gemm        Y = X W_hat^T on the packed 4-bit layer for prefill-sized batches
  *   gptq_gemm_f32            C = alpha op(A) op(B) + beta C at fp32 accuracy: the product kernel
  *                            of prepare and of the lazy block update, exposed on its own
  *   gptq_quantize_layer_noalloc  gptq_quantize_layer on a fixed device scratch array
@@ -285,11 +286,46 @@ const char* gptq_status_string(int status);
  *   batch       1 .. 8
  *   Y           fp32 [batch, ldy], ldy >= d_out (written, not accumulated into)
  * Returns GPTQ_ERR_INVALID_ARG for any other shape, alignment or parameter combination.
+ * With contiguous groups of whole 128-column chunks (or one group per row), d_in a multiple of
+ * 128 and no g_idx, the product runs on the tensor cores with every row's work split evenly over
+ * the SMs: Y is zeroed on the stream and the partial sums of a row are added into it by atomic
+ * adds, so the order of those few additions, and the last bits of Y, can differ between calls.
+ * The other cases run one warp per row and are bitwise repeatable.
  */
 int gptq_dequant_gemv(const uint32_t* qweight, int64_t d_out, int64_t d_in, int bits,
                       const uint16_t* scales_f16, const uint16_t* zeros_f16, int64_t n_groups,
                       int group_size, const int32_t* g_idx, const uint16_t* X, int64_t batch,
                       int64_t ldx, float* Y, int64_t ldy, gptq_stream_t stream);
+
+/*
+ * gptq_dequant_gemm — Y = X W_hat^T on the packed 4-bit format for any number of activation
+ * rows (the prefill counterpart of gptq_dequant_gemv), on the tensor cores.
+ *   "GPTQ: Mathematical Foundations ...", §Inference Execution and Modern Kernel Architectures:
+ *   packed codes are unpacked and dequantized on chip, w_hat = (q - z) * s with the FP16 scale
+ *   and zero, and multiplied with FP16 activations, accumulating in higher precision.
+ *   Y[i, r] = sum_c (code[r, c] - z[r, G(c)]) * s[r, G(c)] * X[i, c] in fp32, computed as
+ *   sum_g s (sum_{c in g} X code - z sum_{c in g} X): the products of activations and codes are
+ *   exact, and every 128 columns the fp32 partial sums are scaled and added in registers.
+ *
+ *   qweight     uint32 [d_out, d_in / 8], the layout gptq_pack writes for 4-bit codes;
+ *               16-byte aligned
+ *   d_in        a multiple of 128
+ *   scales_f16, zeros_f16  fp16 bit patterns [d_out, n_groups]; zero points are integers (other
+ *               values are rounded to one)
+ *   group_size  -1 (n_groups == 1) or a multiple of 128 dividing d_in (n_groups == d_in /
+ *               group_size); act-order g_idx layouts are not taken
+ *   X           fp16 bit patterns [m, ldx], 16-byte aligned, ldx a multiple of 8 and >= d_in
+ *   m           number of activation rows, >= 1
+ *   Y           fp32 [m, ldy], ldy >= d_out (written, not accumulated into)
+ *   dev_status  as for the other calls: work is skipped if it already holds an error, and a
+ *               wait that runs out records GPTQ_ERR_TIMEOUT (then Y holds no result)
+ * Returns GPTQ_ERR_INVALID_ARG for any other shape, alignment or parameter combination.
+ * Results are bitwise repeatable.
+ */
+int gptq_dequant_gemm(const uint32_t* qweight, int64_t d_out, int64_t d_in,
+                      const uint16_t* scales_f16, const uint16_t* zeros_f16, int64_t n_groups,
+                      int group_size, const uint16_t* X, int64_t m, int64_t ldx, float* Y,
+                      int64_t ldy, int32_t* dev_status, gptq_stream_t stream);
 
 /*
  * gptq_gemm_f32 — C = alpha * op(A) * op(B) + beta * C in fp32, the product that

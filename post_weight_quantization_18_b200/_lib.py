@@ -33,7 +33,7 @@ GPTQ_ORDER_GIVEN = 2
 EXPORTED = ("gptq_workspace_size", "gptq_hessian_accumulate", "gptq_prepare_hinv",
             "gptq_quantize_layer", "gptq_pack", "rtn_quantize", "gptq_status_string",
             "gptq_quantize_layer_noalloc", "gptq_dequant_gemv", "gptq_gemm_f32",
-            "gptq_quantize_pack_layer")
+            "gptq_quantize_pack_layer", "gptq_dequant_gemm")
 GPTQ_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -82,6 +82,8 @@ def _load() -> ctypes.CDLL:
     lib.rtn_quantize.restype = I32
     lib.gptq_dequant_gemv.argtypes = [P, I64, I64, I32, P, P, I64, I32, P, P, I64, I64, P, I64, P]
     lib.gptq_dequant_gemv.restype = I32
+    lib.gptq_dequant_gemm.argtypes = [P, I64, I64, P, P, I64, I32, P, I64, I64, P, I64, P, P]
+    lib.gptq_dequant_gemm.restype = I32
     lib.gptq_gemm_f32.argtypes = [I64, I64, I64, F32, P, I64, I32, P, I64, I32, F32, P, I64, P, P]
     lib.gptq_gemm_f32.restype = I32
     lib.gptq_quantize_pack_layer.argtypes = [P, I32, I64, I64, I64, P, P, P, PP, P, P, P, P, P, P,
@@ -276,6 +278,26 @@ def gptq_dequant_gemv(qweight: torch.Tensor, d_in: int, bits: int, scales_f16: t
                                 _ptr(X2), X2.shape[0], X2.stride(0), _ptr(Y2), Y2.stride(0),
                                 _stream())
     _check(rc, "gptq_dequant_gemv")
+
+
+def gptq_dequant_gemm(qweight: torch.Tensor, d_in: int, scales_f16: torch.Tensor,
+                      zeros_f16: torch.Tensor, group_size: int, X: torch.Tensor, Y: torch.Tensor,
+                      dev_status: torch.Tensor | None = None) -> None:
+    """Y [m, d_out] (fp32) = X [m, d_in] (fp16) @ W_hat^T from the packed 4-bit layer."""
+    for t, nm in ((qweight, "qweight"), (scales_f16, "scales_f16"), (zeros_f16, "zeros_f16"),
+                  (X, "X"), (Y, "Y")):
+        _dev(t, nm)
+    if X.dtype != torch.float16 or Y.dtype != torch.float32:
+        raise ValueError("X must be float16 and Y float32")
+    X2 = X.reshape(-1, X.shape[-1])
+    Y2 = Y.reshape(-1, Y.shape[-1])
+    _row_major(X2, "X")
+    _row_major(Y2, "Y")
+    rc = _lib.gptq_dequant_gemm(_ptr(qweight), qweight.shape[0], int(d_in), _ptr(scales_f16),
+                                _ptr(zeros_f16), scales_f16.shape[1], int(group_size), _ptr(X2),
+                                X2.shape[0], X2.stride(0), _ptr(Y2), Y2.stride(0),
+                                _ptr(dev_status), _stream())
+    _check(rc, "gptq_dequant_gemm")
 
 
 def rtn_quantize(W: torch.Tensor, params: gptq_params, codes: torch.Tensor, scales: torch.Tensor,

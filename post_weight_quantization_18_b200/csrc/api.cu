@@ -608,6 +608,33 @@ int gptq_dequant_gemv(const uint32_t* qweight, int64_t d_out, int64_t d_in, int 
              : GPTQ_OK;
 }
 
+int gptq_dequant_gemm(const uint32_t* qweight, int64_t d_out, int64_t d_in,
+                      const uint16_t* scales_f16, const uint16_t* zeros_f16, int64_t n_groups,
+                      int group_size, const uint16_t* X, int64_t m, int64_t ldx, float* Y,
+                      int64_t ldy, int32_t* dev_status, gptq_stream_t stream) {
+  if (qweight == nullptr || scales_f16 == nullptr || zeros_f16 == nullptr || X == nullptr ||
+      Y == nullptr)
+    return GPTQ_ERR_INVALID_ARG;
+  if (d_out < 1 || d_in < 128 || d_in % 128 != 0 || d_in > (1 << 30) || d_out > (1 << 30) ||
+      m < 1 || m > (1 << 30))
+    return GPTQ_ERR_INVALID_ARG;
+  if (ldx < d_in || ldx % 8 != 0 || ldy < d_out) return GPTQ_ERR_INVALID_ARG;
+  if (!aligned(qweight, 16) || !aligned(X, 16) || !aligned(Y, 4) || !aligned(scales_f16, 2) ||
+      !aligned(zeros_f16, 2))
+    return GPTQ_ERR_INVALID_ARG;
+  if (group_size == -1) {
+    if (n_groups != 1) return GPTQ_ERR_INVALID_ARG;
+  } else if (group_size < 128 || group_size % 128 != 0 || d_in % group_size != 0 ||
+             n_groups != d_in / group_size) {
+    return GPTQ_ERR_INVALID_ARG;
+  }
+  return gptq_host::dequant_gemm(qweight, (int)d_out, (int)d_in, scales_f16, zeros_f16,
+                                 (int)n_groups, group_size, X, (int)m, ldx, Y, ldy, dev_status,
+                                 reinterpret_cast<cudaStream_t>(stream))
+             ? GPTQ_ERR_CUDA
+             : GPTQ_OK;
+}
+
 int gptq_gemm_f32(int64_t M, int64_t N, int64_t K, float alpha, const float* A, int64_t lda,
                   int trans_a, const float* B, int64_t ldb, int trans_b, float beta, float* C,
                   int64_t ldc, int32_t* dev_status, gptq_stream_t stream) {

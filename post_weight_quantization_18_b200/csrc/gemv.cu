@@ -36,6 +36,7 @@
 #include <cuda_fp16.h>
 
 #include "common.cuh"
+#include "gemv_pairs.cuh"
 #include "kernels.h"
 
 namespace {
@@ -199,6 +200,10 @@ __device__ __forceinline__ void load_stream(const uint32_t* __restrict__ src, ui
   if constexpr (BITS == 2) {
     asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
                  : "=r"(w[0]), "=r"(w[1]) : "l"(src));
+  } else if constexpr (BITS == 3) {  // a lane's run starts on a 12-byte boundary
+#pragma unroll
+    for (int i = 0; i < 3; ++i)
+      asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(w[i]) : "l"(src + i));
   } else {
 #pragma unroll
     for (int i = 0; i < BITS; i += 4)
@@ -208,199 +213,211 @@ __device__ __forceinline__ void load_stream(const uint32_t* __restrict__ src, ui
   }
 }
 
-// Decoding a word without a shift per pair: a field of BITS bits at bit position pos of both
-// 16-bit halves, or'ed into 0x6400, is the fp16 value 1024 + code * 2^pos as long as
-// pos + BITS <= 10 (it stays in the mantissa). POS_PER_SHIFT fields fit; one shift of the word
-// serves the next POS_PER_SHIFT pairs. fma(v, 2^-pos, -(1024 * 2^-pos + z)) is then code - z,
-// exact in fp16 (a single rounding of an integer below 2^11).
-template <int BITS>
-struct Decode {
-  static constexpr int CPW = 32 / BITS;                 // codes per word
-  static constexpr int PAIRS = CPW / 2;                 // fp16 pairs per word
-  static constexpr int POS_PER_SHIFT = (10 - BITS) / BITS + 1;
-  static constexpr int NPOS = POS_PER_SHIFT < PAIRS ? POS_PER_SHIFT : PAIRS;
-  static constexpr int shift(int j) { return BITS * POS_PER_SHIFT * (j / POS_PER_SHIFT); }
-  static constexpr int pos(int j) { return BITS * (j % POS_PER_SHIFT); }
-};
-
-// Per-row constants -(1024 * 2^-pos + z) for the NPOS field positions, as fp16 pairs (exact:
-// z is an integer below 2^BITS).
-template <int BITS>
-__device__ __forceinline__ void row_consts(__half z, __half2 (&c)[Decode<BITS>::NPOS]) {
-#pragma unroll
-  for (int k = 0; k < Decode<BITS>::NPOS; ++k) {
-    const float off = 1024.f / (float)(1 << (BITS * k));
-    c[k] = __half2half2(__hsub(__float2half_rn(-off), z));
+// The activations of pair P's two columns as an fp16 pair (xr: the run's 32 halves, two per
+// word), in the pairing of gemv_pairs.cuh.
+template <int BITS, int P>
+__device__ __forceinline__ uint32_t pair_x(const uint32_t (&xr)[16]) {
+  constexpr gptq::PairDesc d = gptq::PairSet<BITS>::pair(P);
+  if constexpr (d.j2 == d.j1 + 1 && (d.j1 & 1) == 0) {
+    return xr[d.j1 >> 1];
+  } else {
+    constexpr uint32_t lo = (d.j1 & 1) ? 0x32u : 0x10u;
+    constexpr uint32_t hi = (d.j2 & 1) ? 0x7600u : 0x5400u;
+    return __byte_perm(xr[d.j1 >> 1], xr[d.j2 >> 1], hi | lo);
   }
 }
 
-template <int BITS, int J>
-__device__ __forceinline__ uint32_t pair_minus_z(uint32_t w,
-                                                 const __half2 (&c)[Decode<BITS>::NPOS]) {
-  using D = Decode<BITS>;
-  constexpr int sh = D::shift(J), pos = D::pos(J);
-  constexpr uint32_t m = ((1u << BITS) - 1u) << pos;
-  const uint32_t v = ((w >> sh) & (m | (m << 16))) | 0x64006400u;
-  const __half2 scale = __float2half2_rn(1.f / (float)(1 << pos));
-  const __half2 h =
-      __hfma2(*reinterpret_cast<const __half2*>(&v), scale, c[J % D::POS_PER_SHIFT]);
-  return *reinterpret_cast<const uint32_t*>(&h);
-}
-
-// Word I of the lane's share of a chunk: CPW/4 k-steps. Pair 2s fills k slots 2t, 2t+1 and pair
-// 2s+1 slots 2t+8, 2t+9; the activations of those columns are paired the same way.
-template <int BITS, int I, int S = 0>
-__device__ __forceinline__ void word_steps(uint32_t wa, uint32_t wb, const uint32_t (&xr)[16],
-                                           const __half2 (&ca)[Decode<BITS>::NPOS],
-                                           const __half2 (&cb)[Decode<BITS>::NPOS],
-                                           float (&d0)[4], float (&d1)[4]) {
-  constexpr int CPW = Decode<BITS>::CPW;
-  if constexpr (S < CPW / 4) {
-    const uint32_t a0 = pair_minus_z<BITS, 2 * S>(wa, ca);
-    const uint32_t a1 = pair_minus_z<BITS, 2 * S>(wb, cb);
-    const uint32_t a2 = pair_minus_z<BITS, 2 * S + 1>(wa, ca);
-    const uint32_t a3 = pair_minus_z<BITS, 2 * S + 1>(wb, cb);
-    constexpr int r = I * CPW / 2 + S;
-    const uint32_t b0 = __byte_perm(xr[r], xr[r + CPW / 4], 0x5410);
-    const uint32_t b1 = __byte_perm(xr[r], xr[r + CPW / 4], 0x7632);
-    if constexpr (((I * (CPW / 4) + S) & 1) == 0)
-      mma_16816(d0, a0, a1, a2, a3, b0, b1);
-    else
-      mma_16816(d1, a0, a1, a2, a3, b0, b1);
-    word_steps<BITS, I, S + 1>(wa, wb, xr, ca, cb, d0, d1);
+template <int BITS, int Q = 0>
+__device__ __forceinline__ void act_pairs(const uint32_t (&xr)[16], uint32_t (&b)[16]) {
+  if constexpr (Q < 16) {
+    b[Q] = pair_x<BITS, Q>(xr);
+    act_pairs<BITS, Q + 1>(xr, b);
   }
 }
 
-template <int BITS, int I = 0>
-__device__ __forceinline__ void chunk_words(const uint32_t (&wa)[BITS],
-                                            const uint32_t (&wb)[BITS], const uint32_t (&xr)[16],
-                                            const __half2 (&ca)[Decode<BITS>::NPOS],
-                                            const __half2 (&cb)[Decode<BITS>::NPOS],
-                                            float (&d0)[4], float (&d1)[4]) {
-  if constexpr (I < BITS) {
-    word_steps<BITS, I>(wa[I], wb[I], xr, ca, cb, d0, d1);
-    chunk_words<BITS, I + 1>(wa, wb, xr, ca, cb, d0, d1);
+// The 8 MMAs of one m-tile and chunk: rows g (words wa) and g + 8 (words wb).
+template <int BITS, int Q = 0>
+__device__ __forceinline__ void tile_mmas(const uint32_t (&wa)[BITS], const uint32_t (&wb)[BITS],
+                                          const uint32_t (&b)[16],
+                                          float (&dc)[gptq::PairSet<BITS>::NCLS][4]) {
+  if constexpr (Q < 8) {
+    using gptq::pair_code;
+    mma_16816(dc[gptq::PairSet<BITS>::cls(Q)], pair_code<BITS>(wa, 2 * Q),
+              pair_code<BITS>(wb, 2 * Q), pair_code<BITS>(wa, 2 * Q + 1),
+              pair_code<BITS>(wb, 2 * Q + 1), b[2 * Q], b[2 * Q + 1]);
+    tile_mmas<BITS, Q + 1>(wa, wb, b, dc);
   }
 }
 
-// Group parameters of rows g and g + 8.
-struct GroupParams {
-  __half sa, sb, za, zb;
-};
+// Work items are (row tile, chunk) pairs, a row tile being MT m-tiles of 16 rows: the activation
+// pairs and the all-ones MMAs of a chunk serve every m-tile. The grid is persistent (every CTA
+// resident at once) and the items, in tile-major order, are split evenly over the CTAs and then
+// over each CTA's warps, so every SM gets the same work whatever the row count; a warp that
+// finishes a row tile (or its range) adds its partial sums into Y, which the launcher zeroes.
+// The warps run independently (no barrier), each with a ring of 2 items' packed words per row.
+// (Measured on B200 at 8192 x 28672, 4-bit, batch 1: 42.9 us; one producer warp per CTA
+// preparing the activation pairs for 4 to 8 lock-stepped consumer warps through shared memory:
+// 57 to 67 us.)
+constexpr int kTcWarps = 8;
 
-// The ring holds 2 * BURST chunks of packed words per lane; BURST consecutive chunks (BURST *
-// 64 contiguous bytes of a row for 4-bit codes) are requested back to back. Measured on B200 at
-// 8192 x 28672, 4-bit: BURST 1 (76 registers, six warps per CTA, one wave) beats BURST 2
-// (98 registers, fewer warps) and a forced 80-register BURST 2 (spills).
-template <int BITS, int BURST>
-__global__ void __launch_bounds__(kMmaMaxWarps * 32)
-dequant_gemv_mma_kernel(const uint32_t* __restrict__ qweight, int n, int d, long long wpr,
-                        const __half* __restrict__ scales, const __half* __restrict__ zeros,
-                        int G, int chunks_per_group, const __half* __restrict__ X, long long ldx,
-                        int batch, float* __restrict__ Y, long long ldy) {
-  using D = Decode<BITS>;
-  __shared__ float4 red[kMmaMaxWarps][32];
+// Row r of this lane in row tile `tile`: m-tile r / 2, half r % 2. Rows past the end read the
+// last row (valid memory) and are not written.
+template <int MT>
+__device__ __forceinline__ int lane_row(int tile, int r, int g, int n) {
+  return min(tile * 16 * MT + 16 * (r >> 1) + g + 8 * (r & 1), n - 1);
+}
+
+template <int BITS, int MT>
+__global__ void __launch_bounds__(kTcWarps * 32)
+dequant_gemv_tc_kernel(const uint32_t* __restrict__ qweight, int n, int d, long long wpr,
+                       const __half* __restrict__ scales, const __half* __restrict__ zeros, int G,
+                       int chunks_per_group, const __half* __restrict__ X, long long ldx,
+                       int batch, float* __restrict__ Y, long long ldy) {
+  using PS = gptq::PairSet<BITS>;
+  constexpr int NR = 2 * MT;                // rows per lane: m-tile m, half h -> 2 m + h
+  constexpr int CW = kChunk * BITS / 32;    // words of one row in a chunk
+  // sum(code * x) = sum_c 2^(24 - pos_c) d_c; with two classes 2^20 (16 d_0 + d_1).
+  constexpr float kScale = PS::NCLS == 2 ? 1048576.f : 16777216.f;
   const int nw = blockDim.x >> 5;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
-  const int row0 = blockIdx.x * 16;
-  // Rows past the end read the last row (valid memory) and are not written; batch rows past the
-  // batch read the last batch row and land in accumulator columns that are not written.
-  const int ra = min(row0 + g, n - 1), rb = min(row0 + g + 8, n - 1);
   const int chunks = d / kChunk;
-  const int c_begin = (int)((long long)chunks * warp / nw);
-  const int c_end = (int)((long long)chunks * (warp + 1) / nw);
-  const int nc = c_end - c_begin;
-  constexpr int CW = kChunk * BITS / 32;  // words of one row in a chunk
-  const uint32_t* pa = qweight + (long long)ra * wpr + t * BITS + (long long)c_begin * CW;
-  const uint32_t* pb = qweight + (long long)rb * wpr + t * BITS + (long long)c_begin * CW;
-  const __half* xp =
-      X + (long long)min(g, batch - 1) * ldx + 32 * t + (long long)c_begin * kChunk;
-  const __half* sa = scales + (long long)ra * G;
-  const __half* sb = scales + (long long)rb * G;
-  const __half* za = zeros + (long long)ra * G;
-  const __half* zb = zeros + (long long)rb * G;
+  const long long items = (long long)((n + 16 * MT - 1) / (16 * MT)) * chunks;
+  const long long c0 = items * blockIdx.x / gridDim.x, c1 = items * (blockIdx.x + 1) / gridDim.x;
+  const long long i_begin = c0 + (c1 - c0) * warp / nw;
+  const long long i_end = c0 + (c1 - c0) * (warp + 1) / nw;
+  if (i_begin >= i_end) return;
+  // Batch rows past the batch read the last batch row and land in accumulator columns that are
+  // not written.
+  const __half* xrow = X + (long long)min(g, batch - 1) * ldx + 32 * t;
 
-  uint32_t wa[2][BURST][BITS], wb[2][BURST][BITS];
+  // Position of the current item, and of the item the next prefetch loads (pw: its rows'
+  // packed words at chunk 0, this lane's run).
+  int tile = (int)(i_begin / chunks), chunk = (int)(i_begin % chunks);
+  int p_tile = tile, p_chunk = chunk;
+  const uint32_t* pw[NR];
+  auto set_prefetch_rows = [&]() {
 #pragma unroll
-  for (int h = 0; h < 2; ++h)
+    for (int r = 0; r < NR; ++r)
+      pw[r] = qweight + (long long)lane_row<MT>(p_tile, r, g, n) * wpr + t * BITS;
+  };
+  set_prefetch_rows();
+  uint32_t wr[2][NR][BITS];
 #pragma unroll
-    for (int k = 0; k < BURST; ++k)
-      if (h * BURST + k < nc) {
-        load_stream<BITS>(pa + (h * BURST + k) * CW, wa[h][k]);
-        load_stream<BITS>(pb + (h * BURST + k) * CW, wb[h][k]);
+  for (int h = 0; h < 2; ++h) {
+    if (i_begin + h < i_end) {
+#pragma unroll
+      for (int r = 0; r < NR; ++r) load_stream<BITS>(pw[r] + (long long)p_chunk * CW, wr[h][r]);
+    }
+    if (++p_chunk == chunks) {
+      p_chunk = 0;
+      ++p_tile;
+      set_prefetch_rows();
+    }
+  }
+
+  // Group bookkeeping without a division per chunk (one per tile change); the next group's
+  // parameters are fetched when a group starts.
+  int gi = 0, g_next = 0;
+  __half nxt_s[NR], nxt_z[NR];
+  float sc[NR], nsz[NR];  // s * 2^(24 - pos): the scale of the class sums; -s * z
+  long long poff[NR];     // row * G of the current tile's rows
+  auto start_tile = [&]() {
+    gi = min(chunk / chunks_per_group, G - 1);
+    g_next = (gi + 1) * chunks_per_group;
+#pragma unroll
+    for (int r = 0; r < NR; ++r) {
+      poff[r] = (long long)lane_row<MT>(tile, r, g, n) * G;
+      // zero points are integers; another value is rounded to one, as the other paths do
+      const float sv = __half2float(scales[poff[r] + gi]);
+      const float zv = rintf(__half2float(zeros[poff[r] + gi]));
+      sc[r] = sv * kScale;
+      nsz[r] = -sv * zv;
+      nxt_s[r] = scales[poff[r] + min(gi + 1, G - 1)];
+      nxt_z[r] = zeros[poff[r] + min(gi + 1, G - 1)];
+    }
+  };
+  start_tile();
+
+  float acc[MT][4];
+#pragma unroll
+  for (int m = 0; m < MT; ++m) acc[m][0] = acc[m][1] = acc[m][2] = acc[m][3] = 0.f;
+  // Accumulator layout: element e is (row g + 8 (e >> 1), batch column 2t + (e & 1)).
+  auto flush = [&]() {
+#pragma unroll
+    for (int m = 0; m < MT; ++m)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int bcol = 2 * t + (e & 1);
+        const int row = tile * 16 * MT + 16 * m + g + 8 * (e >> 1);
+        if (bcol < batch && row < n) atomicAdd(Y + (long long)bcol * ldy + row, acc[m][e]);
+        acc[m][e] = 0.f;
       }
-
-  // Group bookkeeping without a division per chunk; the next group's parameters are fetched
-  // when a group starts. (A warp with no chunks reads group 0, which exists.)
-  int gi = c_begin / chunks_per_group;
-  if (gi >= G) gi = G - 1;
-  int g_next = (gi + 1) * chunks_per_group;  // first chunk of the next group
-  GroupParams cur{sa[gi], sb[gi], za[gi], zb[gi]};
-  GroupParams nxt = cur;
-  if (gi + 1 < G) nxt = GroupParams{sa[gi + 1], sb[gi + 1], za[gi + 1], zb[gi + 1]};
-  __half2 ca[D::NPOS], cb[D::NPOS];
-  row_consts<BITS>(cur.za, ca);
-  row_consts<BITS>(cur.zb, cb);
-  float s_a = __half2float(cur.sa), s_b = __half2float(cur.sb);
-
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int base = 0; base < nc; base += 2 * BURST) {
+  };
+  const uint32_t ones = 0x3C003C00u;  // fp16 (1, 1)
+  for (long long it = i_begin; it < i_end; it += 2) {
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
+      if (it + h < i_end) {
+        if (chunk == g_next) {
+          ++gi;
+          g_next += chunks_per_group;
 #pragma unroll
-      for (int k = 0; k < BURST; ++k) {
-        const int ci = base + h * BURST + k;
-        if (ci < nc) {
-          if (c_begin + ci == g_next) {
-            ++gi;
-            g_next += chunks_per_group;
-            cur = nxt;
-            if (gi + 1 < G) nxt = GroupParams{sa[gi + 1], sb[gi + 1], za[gi + 1], zb[gi + 1]};
-            row_consts<BITS>(cur.za, ca);
-            row_consts<BITS>(cur.zb, cb);
-            s_a = __half2float(cur.sa);
-            s_b = __half2float(cur.sb);
+          for (int r = 0; r < NR; ++r) {
+            const float sv = __half2float(nxt_s[r]), zv = rintf(__half2float(nxt_z[r]));
+            sc[r] = sv * kScale;
+            nsz[r] = -sv * zv;
+            nxt_s[r] = scales[poff[r] + min(gi + 1, G - 1)];
+            nxt_z[r] = zeros[poff[r] + min(gi + 1, G - 1)];
           }
-          uint32_t xr[16];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint4 v = __ldg(reinterpret_cast<const uint4*>(xp + ci * kChunk) + i);
-            xr[4 * i] = v.x; xr[4 * i + 1] = v.y; xr[4 * i + 2] = v.z; xr[4 * i + 3] = v.w;
-          }
-          float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
-          chunk_words<BITS>(wa[h][k], wb[h][k], xr, ca, cb, d0, d1);
-          acc[0] = fmaf(s_a, d0[0] + d1[0], acc[0]);
-          acc[1] = fmaf(s_a, d0[1] + d1[1], acc[1]);
-          acc[2] = fmaf(s_b, d0[2] + d1[2], acc[2]);
-          acc[3] = fmaf(s_b, d0[3] + d1[3], acc[3]);
         }
-      }
+        uint32_t xr[16];
 #pragma unroll
-      for (int k = 0; k < BURST; ++k) {
-        const int cn = base + (h + 2) * BURST + k;
-        if (cn < nc) {
-          load_stream<BITS>(pa + cn * CW, wa[h][k]);
-          load_stream<BITS>(pb + cn * CW, wb[h][k]);
+        for (int i = 0; i < 4; ++i) {
+          const uint4 v = __ldg(reinterpret_cast<const uint4*>(xrow + (long long)chunk * kChunk) + i);
+          xr[4 * i] = v.x; xr[4 * i + 1] = v.y; xr[4 * i + 2] = v.z; xr[4 * i + 3] = v.w;
+        }
+        uint32_t b[16];
+        act_pairs<BITS>(xr, b);
+        float dx[4] = {0.f, 0.f, 0.f, 0.f};  // the chunk's sum of x per batch column
+#pragma unroll
+        for (int q = 0; q < 8; ++q) mma_16816(dx, ones, ones, ones, ones, b[2 * q], b[2 * q + 1]);
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          float dc[PS::NCLS][4];
+#pragma unroll
+          for (int c = 0; c < PS::NCLS; ++c) dc[c][0] = dc[c][1] = dc[c][2] = dc[c][3] = 0.f;
+          tile_mmas<BITS>(wr[h][2 * m], wr[h][2 * m + 1], b, dc);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float cx = PS::NCLS == 2 ? fmaf(16.f, dc[0][e], dc[1][e]) : dc[0][e];
+            const int r = 2 * m + (e >> 1);
+            acc[m][e] = fmaf(sc[r], cx, acc[m][e]);
+            acc[m][e] = fmaf(nsz[r], dx[e], acc[m][e]);
+          }
+        }
+        // Refill this ring slot with the item two ahead.
+        if (it + h + 2 < i_end) {
+#pragma unroll
+          for (int r = 0; r < NR; ++r)
+            load_stream<BITS>(pw[r] + (long long)p_chunk * CW, wr[h][r]);
+        }
+        if (++p_chunk == chunks) {
+          p_chunk = 0;
+          ++p_tile;
+          set_prefetch_rows();
+        }
+        // Next item.
+        if (++chunk == chunks) {
+          flush();
+          chunk = 0;
+          ++tile;
+          if (it + h + 1 < i_end) start_tile();
         }
       }
     }
   }
-  red[warp][lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-  __syncthreads();
-  if (warp != 0) return;
-  for (int w = 1; w < nw; ++w) {
-    const float4 v = red[w][lane];
-    acc[0] += v.x; acc[1] += v.y; acc[2] += v.z; acc[3] += v.w;
-  }
-  // Accumulator layout: acc[e] is (row g, batch 2t + e), acc[2 + e] is (row g + 8, batch 2t + e).
-#pragma unroll
-  for (int e = 0; e < 2; ++e) {
-    const int b = 2 * t + e;
-    if (b >= batch) continue;
-    if (row0 + g < n) Y[(long long)b * ldy + row0 + g] = acc[e];
-    if (row0 + g + 8 < n) Y[(long long)b * ldy + row0 + g + 8] = acc[2 + e];
-  }
+  if (chunk != 0) flush();
 }
 
 }  // namespace
@@ -409,28 +426,24 @@ namespace gptq_host {
 
 namespace {
 
-// Warps per CTA for the tensor-core kernel: the most of 8, 6 or 4 that still lets every 16-row
-// tile be resident at once (one wave); 4 when no choice fits.
+// The tensor-core kernel runs persistent: kTcWarps warps per CTA and as many CTAs as are
+// resident at once (at most one per 16 work items), each taking an even share of the items. Y is
+// zeroed first: the warps add their partial sums into it.
 template <class K>
-int mma_launch(K kernel, int tiles, const uint32_t* qweight, int n, int d, long long wpr,
-               const __half* s, const __half* z, int G, int cpg, const __half* x, long long ldx,
-               int batch, float* y, long long ldy, cudaStream_t stream) {
-  int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+int tc_launch(K kernel, long long items, const uint32_t* qweight, int n, int d, long long wpr,
+              const __half* s, const __half* z, int G, int cpg, const __half* x, long long ldx,
+              int batch, float* y, long long ldy, cudaStream_t stream) {
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kTcWarps * 32, 0) !=
+      cudaSuccess)
     return GPTQ_ERR_CUDA;
-  int nw = 4;
-  for (int cand : {8, 6}) {
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, cand * 32, 0) !=
-        cudaSuccess)
-      return GPTQ_ERR_CUDA;
-    if ((long long)per_sm * sms >= tiles) {
-      nw = cand;
-      break;
-    }
-  }
-  kernel<<<tiles, nw * 32, 0, stream>>>(qweight, n, d, wpr, s, z, G, cpg, x, ldx, batch, y, ldy);
+  long long grid = (long long)num_sms() * (per_sm > 0 ? per_sm : 1);
+  if (grid > (items + 15) / 16) grid = (items + 15) / 16;
+  if (cudaMemset2DAsync(y, (size_t)ldy * 4, 0, (size_t)n * 4, (size_t)batch, stream) !=
+      cudaSuccess)
+    return GPTQ_ERR_CUDA;
+  kernel<<<(int)grid, kTcWarps * 32, 0, stream>>>(qweight, n, d, wpr, s, z, G, cpg, x, ldx, batch,
+                                                   y, ldy);
   return cudaGetLastError() == cudaSuccess ? 0 : GPTQ_ERR_CUDA;
 }
 
@@ -450,19 +463,22 @@ int dequant_gemv(const uint32_t* qweight, int n, int d, int bits, const uint16_t
                                                                group_size, g_idx, x, ldx, batch,   \
                                                                y, ldy)
   const bool run_groups = g_idx == nullptr && (n_groups == 1 || group_size % kChunk == 0);
-  if (run_groups && d % kChunk == 0 && (bits == 2 || bits == 4 || bits == 8)) {
-    const int tiles = (n + 15) / 16;
+  if (run_groups && d % kChunk == 0 && (bits == 2 || bits == 3 || bits == 4 || bits == 8)) {
     const int cpg = n_groups == 1 ? d / kChunk : group_size / kChunk;
+    auto items = [&](int mt) { return (long long)((n + 16 * mt - 1) / (16 * mt)) * (d / kChunk); };
     switch (bits) {
       case 2:
-        return mma_launch(dequant_gemv_mma_kernel<2, 2>, tiles, qweight, n, d, wpr, s, z,
-                          n_groups, cpg, x, ldx, batch, y, ldy, stream);
+        return tc_launch(dequant_gemv_tc_kernel<2, 2>, items(2), qweight, n, d, wpr, s, z,
+                         n_groups, cpg, x, ldx, batch, y, ldy, stream);
+      case 3:
+        return tc_launch(dequant_gemv_tc_kernel<3, 2>, items(2), qweight, n, d, wpr, s, z,
+                         n_groups, cpg, x, ldx, batch, y, ldy, stream);
       case 4:
-        return mma_launch(dequant_gemv_mma_kernel<4, 1>, tiles, qweight, n, d, wpr, s, z,
-                          n_groups, cpg, x, ldx, batch, y, ldy, stream);
+        return tc_launch(dequant_gemv_tc_kernel<4, 2>, items(2), qweight, n, d, wpr, s, z,
+                         n_groups, cpg, x, ldx, batch, y, ldy, stream);
       default:
-        return mma_launch(dequant_gemv_mma_kernel<8, 1>, tiles, qweight, n, d, wpr, s, z,
-                          n_groups, cpg, x, ldx, batch, y, ldy, stream);
+        return tc_launch(dequant_gemv_tc_kernel<8, 1>, items(1), qweight, n, d, wpr, s, z,
+                         n_groups, cpg, x, ldx, batch, y, ldy, stream);
     }
   }
   const bool one = batch == 1;

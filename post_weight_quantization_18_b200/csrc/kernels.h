@@ -111,6 +111,11 @@ int dequant_gemv(const uint32_t* qweight, int n, int d, int bits, const uint16_t
                  const uint16_t* zeros_f16, int n_groups, int group_size, const int32_t* g_idx,
                  const uint16_t* x_f16, int batch, long long ldx, float* y, long long ldy,
                  cudaStream_t stream);
+// Y [m, ldy] = X [m, ldx] W_hat^T on the packed 4-bit format, tcgen05 (dequant_gemm.cu).
+int dequant_gemm(const uint32_t* qweight, int n, int d, const uint16_t* scales_f16,
+                 const uint16_t* zeros_f16, int n_groups, int group_size, const uint16_t* x_f16,
+                 int m, long long ldx, float* y, long long ldy, const int32_t* status,
+                 cudaStream_t stream);
 
 // ---- RTN and pack ----
 int rtn_launch(const void* W, int w_dtype, long long ldw, int n, int d, int bits, int group_size,

@@ -61,6 +61,13 @@ int main(void) {
                           fake_f, 64, NULL) == GPTQ_ERR_INVALID_ARG,
         "gemv: batch above 8");
 
+  check(gptq_dequant_gemm(fake_q, 64, 192, fake_h, fake_h, 1, -1, fake_h, 16, 192, fake_f, 64,
+                          NULL, NULL) == GPTQ_ERR_INVALID_ARG,
+        "dequant gemm: d_in not a multiple of 128");
+  check(gptq_dequant_gemm(fake_q, 64, 256, fake_h, fake_h, 4, 64, fake_h, 16, 256, fake_f, 64,
+                          NULL, NULL) == GPTQ_ERR_INVALID_ARG,
+        "dequant gemm: groups of 64 columns");
+
   check(gptq_gemm_f32(8, 8, 8, 1.0f, fake_f, 8, 0, fake_f, 8, 0, 0.0f, NULL, 8, NULL, NULL) ==
             GPTQ_ERR_INVALID_ARG,
         "gemm: null C");

@@ -25,7 +25,8 @@ def declared_functions():
 
 def test_header_declares_the_boundary():
     assert declared_functions() == sorted([
-        "gptq_dequant_gemv", "gptq_gemm_f32", "gptq_hessian_accumulate", "gptq_pack",
+        "gptq_dequant_gemm", "gptq_dequant_gemv", "gptq_gemm_f32", "gptq_hessian_accumulate",
+        "gptq_pack",
         "gptq_prepare_hinv", "gptq_quantize_pack_layer",
         "gptq_quantize_layer", "gptq_quantize_layer_noalloc", "gptq_status_string",
         "gptq_workspace_size", "rtn_quantize"])
@@ -132,6 +133,31 @@ def test_dequant_gemv_rejects_bad_arguments_on_host(lib):
     assert call(x=V(0x1004)) == 1           # X not 16-byte aligned
     assert call(g=48) == 1                  # group size does not divide d_in
     assert call(G=2) == 1                   # n_groups disagrees with group_size
+    assert call(g=-1, G=2) == 1
+
+
+def test_dequant_gemm_rejects_bad_arguments_on_host(lib):
+    V, I64, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    lib.gptq_dequant_gemm.argtypes = [V, I64, I64, V, V, I64, I, V, I64, I64, V, I64, V, V]
+    lib.gptq_dequant_gemm.restype = I
+    fake = V(0x1000)  # 16-byte aligned, never dereferenced: every call fails its checks
+    ok = dict(q=fake, n=64, d=256, s=fake, z=fake, G=2, g=128, x=fake, m=40, ldx=256, y=fake,
+              ldy=64, st=None, stream=None)
+    names = list(ok)
+
+    def call(**kw):
+        args = dict(ok)
+        args.update(kw)
+        return lib.gptq_dequant_gemm(*[args[k] for k in names])
+
+    assert call(q=None) == 1 and call(x=None) == 1 and call(y=None) == 1
+    assert call(d=192, G=1, g=-1) == 1      # d_in not a multiple of 128
+    assert call(m=0) == 1
+    assert call(ldx=260) == 1               # not a multiple of 8
+    assert call(ldy=63) == 1
+    assert call(x=V(0x1004)) == 1           # X not 16-byte aligned
+    assert call(g=64, G=4) == 1             # groups must be whole multiples of 128 columns
+    assert call(G=3) == 1                   # n_groups disagrees with group_size
     assert call(g=-1, G=2) == 1
 
 

@@ -204,3 +204,30 @@ def test_syrk_unit_order_on_cpu(tmp_path, n_tb, grp, n_split):
     for g in np.unique(grp_id):
         splits = got[grp_id == g, 2]
         assert np.all(np.diff(splits) >= 0)
+
+
+@pytest.mark.skipif(shutil.which("g++") is None, reason="needs g++")
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+def test_gemv_pair_decoding_on_cpu(tmp_path, bits):
+    """The tensor-core GEMV's pair decoding (gemv_pairs.cuh, the functions the kernel calls):
+    every code of a 32-code run, packed by the oracle, comes back once, as a clean in-place field
+    of an fp16 half, at the run column the activation pairing assumes."""
+    import numpy as np
+    from oracle import pack as pk
+    exe = tmp_path / "gemv_pairs_check"
+    r = subprocess.run(["g++", "-std=c++17", "-O2", "-Wall", "-Werror", "-Wno-unknown-pragmas",
+                        "-I", os.path.join(ROOT, "post_weight_quantization_18_b200", "csrc"),
+                        os.path.join(ROOT, "tests", "c", "gemv_pairs_check.cpp"), "-o", str(exe)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    n = 300
+    codes = np.random.default_rng(bits).integers(0, 2 ** bits, (n, 32), dtype=np.uint8)
+    codes[0] = 2 ** bits - 1
+    codes[1] = 0
+    words = pk.pack_rows(codes, bits)               # oracle packing: `bits` words per 32 codes
+    (tmp_path / "in.bin").write_bytes(words.astype(np.uint32).tobytes())
+    r = subprocess.run([str(exe), str(bits), str(n), str(tmp_path / "in.bin"),
+                        str(tmp_path / "out.bin")], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, r.returncode
+    out = np.frombuffer((tmp_path / "out.bin").read_bytes(), np.uint8).reshape(n, 32)
+    np.testing.assert_array_equal(out, codes)

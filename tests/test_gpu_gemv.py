@@ -69,6 +69,11 @@ def _w_hat(qn, sn, zn, gi, d, bits):
     (136, 3072, 2, 128, False, 5),    # 2-bit, odd batch
     (64, 1152, 4, -1, False, 1),      # one group per row, chunk count not a multiple of warps
     (96, 1056, 4, -1, False, 2),      # d_in not a multiple of 128: warp-per-row path
+    # 3-bit codes on the tensor cores: runs of 3 words, pairs straddling word boundaries
+    (1000, 4096, 3, 128, False, 1),
+    (136, 3072, 3, -1, False, 5),
+    (40, 2048, 3, 256, False, 8),     # fewer rows than one CTA's tiles
+    (520, 1024, 2, 128, False, 1),    # 2-bit, ragged last tile
 ])
 def test_dequant_gemv_matches_oracle(n, d, bits, g, perm, batch):
     qw, s16, z16, g_idx, _ = _packed_layer(n, d, bits, g, seed=n + d + bits, gidx_perm=perm)
