@@ -553,9 +553,12 @@ def run_ours(args):
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
+        # An NVTX range marks the timed steps for profilers (ncu --nvtx-include bench_timed/).
+        torch.cuda.nvtx.range_push("bench_timed")
         for _ in range(args.steps):
             flush.zero_()
             step(Xd, Wd, True, graphs)
+        torch.cuda.nvtx.range_pop()
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
