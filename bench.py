@@ -2,9 +2,9 @@
 """Benchmark: GPTQ quantization of one linear layer per step, end to end on the GPU.
 
 A step is the whole hot path for one layer: H = 2 X^T X over all calibration tokens
-(gptq_hessian_accumulate), damping + U = upper Cholesky factor of H^-1 (gptq_prepare_hinv), the
-column sweep with lazy updates (gptq_quantize_layer) and packing (gptq_pack), all through the C
-ABI. Default workload: the largest single-GPU layer, a Llama-70B-shaped down projection,
+(gptq_hessian_accumulate), damping + U = upper Cholesky factor of H^-1 (gptq_prepare_hinv), and
+the column sweep with lazy updates writing the packed layer (gptq_quantize_pack_layer), all
+through the C ABI. Default workload: the largest single-GPU layer, a Llama-70B-shaped down projection,
 W 8192 x 28672 bf16 ~ N(0, 0.015^2), X 131072 x 28672 bf16 half-normal with lognormal(0, 1)
 channel scales and 0.05 % outlier channels x30, 4-bit symmetric with one scale per row,
 block 128, damp 0.01 (a 28672^2 fp32 Hessian). --workload selects another one.
@@ -15,10 +15,12 @@ Prints one JSON line (rank 0). Under torchrun each rank quantizes its own layer 
 problems, no collective on the data path: weak scaling); the timed duration is the max over ranks.
 --impl reference times the FP64 CPU oracle on bounded samples of the same workload.
 Besides the headline the line reports the per-stage times (breakdown_ms) and each stage's
-roofline (stages), the SYRK kernel's roofline (roofline), the end-to-end rate through the C ABI
-from pinned host buffers (e2e), the oracle's rate on the host cores (cpu_baseline), the number
-of kernels launched in the timed steps (counted from the recorded CUDA graphs), and the
-dequantizing GEMV on a packed 8192 x 28672 int4 layer (dequant_gemv).
+roofline (stages), the dominant kernel's roofline (roofline: the 3xTF32 GEMM at the step's
+largest product, timed live) and the SYRK's (roofline_syrk), the end-to-end rate through the C
+ABI from pinned host buffers (e2e: X streamed in chunks whose copies overlap the SYRK), the
+oracle's rate on the host cores (cpu_baseline), the number of kernels launched in the timed
+steps (counted from the recorded CUDA graphs), and the dequantizing GEMV on a packed
+8192 x 28672 int4 layer (dequant_gemv).
 """
 from __future__ import annotations
 
@@ -562,17 +564,38 @@ def run_ours(args):
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
-        # End to end: pinned host inputs -> device -> hot path -> packed result back to host.
+        # End to end: pinned host inputs -> device -> hot path -> packed result back to host,
+        # through the public calls as a user streams calibration data: X arrives in chunks of
+        # whole 8192-token ranges on a copy stream and H accumulates each chunk as it lands
+        # (gptq_hessian_accumulate with accumulate = 1 after the first), so the host-to-device
+        # copies overlap the SYRK; W's copy overlaps prepare, which does not read it.
+        compute = torch.cuda.current_stream()
+        copy_stream = torch.cuda.Stream(device=dev)
+        chunk = max(8192, -(-N // (16 * 8192)) * 8192)
+        bounds = [(t0, min(N, t0 + chunk)) for t0 in range(0, N, chunk)]
         e2e_ev = []
         for _ in range(args.e2e_steps):
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record()
-            Xd.copy_(Xh, non_blocking=True)
-            Wd.copy_(Wh, non_blocking=True)
-            step(Xd, Wd, False)
+            a.record(compute)
+            copy_stream.wait_event(a)
+            landed = []
+            with torch.cuda.stream(copy_stream):
+                for t0, t1 in bounds:
+                    Xd[t0:t1].copy_(Xh[t0:t1], non_blocking=True)
+                    landed.append(torch.cuda.Event())
+                    landed[-1].record(copy_stream)
+                Wd.copy_(Wh, non_blocking=True)
+                w_landed = torch.cuda.Event()
+                w_landed.record(copy_stream)
+            for i, (t0, t1) in enumerate(bounds):
+                compute.wait_event(landed[i])
+                L.gptq_hessian_accumulate(H, Xd[t0:t1], 2.0, i > 0, status)
+            calls[1](Xd, Wd)
+            compute.wait_event(w_landed)
+            calls[2](Xd, Wd)
             for h, t in zip(outs_h, (qweight, s16, z16, g_idx)):
                 h.copy_(t, non_blocking=True)
-            b.record()
+            b.record(compute)
             e2e_ev.append((a, b))
         torch.cuda.synchronize()
     st = status.cpu().tolist()

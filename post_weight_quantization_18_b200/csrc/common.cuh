@@ -98,7 +98,7 @@ GPTQ_DEV void fence_proxy_async_smem() {
 }
 
 // ------------------------------------------------------------------------------------------
-// TMA (cp.async.bulk.tensor) — loads without multicast, reduce-add stores.
+// TMA (cp.async.bulk.tensor): plain tile loads into this CTA, reduce-add stores.
 // ------------------------------------------------------------------------------------------
 GPTQ_DEV void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
