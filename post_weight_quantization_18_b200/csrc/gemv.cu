@@ -9,7 +9,8 @@
 // Y[b, r] = sum_c (code[r, c] - z[r, G(c)]) * s[r, G(c)] * X[b, c], b < batch <= 8, with
 // G(c) = g_idx[c], or c / group_size when g_idx is NULL (0 for one group per row).
 //
-// Layout: one warp per output row. A row of qweight is one LSB-first bit stream along d_in
+// Warp-per-row path (act-order g_idx, groups shorter than 128 columns, d_in not a multiple of
+// 128): one warp per output row. A row of qweight is one LSB-first bit stream along d_in
 // (code k at stream bits [b k, b k + b)); lane l takes runs of 32 codes, i.e. exactly BITS words,
 // run l, l + 32, ..., so a warp reads 128 * BITS contiguous bytes per step (16-byte loads for
 // 4 and 8 bits). The 32 codes of a run come out of the BITS words with compile-time shifts (a
@@ -18,21 +19,17 @@
 // Y += s * sum (q - z) x; otherwise the parameters are looked up per column. Activations are
 // read 8 halves at a time; all sums are fp32, added across the warp with shuffles.
 //
-// Tensor-core path (2-, 4- and 8-bit codes, contiguous groups that are whole multiples of
-// 128 columns or one group per row, d_in a multiple of 128): a CTA owns 16 output rows and its
-// warps split d_in into 128-column chunks. Per chunk a warp issues 8 mma.sync m16n8k16 (fp16 in,
-// fp32 accumulate) with A = code - z (16 rows x 16 columns) and B = X (16 columns x 8 batch
-// rows, zero beyond the batch). Lane (g, t) holds rows g and g + 8 and the 32 columns
-// [32 t, 32 t + 32) of the chunk, which are exactly `bits` packed words per row. Because the
-// dot product sums over columns, the order in which those 32 columns enter the MMA's k slots is
-// free as long as A and B use the same one: a word of 32 / bits codes gives the fp16 pairs
-// (code j, code j + 16 / bits) with one mask-and-or, 0x6400 | (code << pos) being the fp16
-// value 1024 + code * 2^pos, and one half2 fma with 2^-pos and -(1024 * 2^-pos + z) leaves
-// code - z exactly (integers below 2^11); a shift of the word is needed only once the field
-// would leave the 10-bit mantissa. The activations take the same pairing with byte permutes.
-// Warps per CTA (4, 6 or 8) are the most that keep every tile resident. The 8 k-steps of a chunk
-// accumulate in fp32 on the tensor core; the chunk's sum is then scaled by its group's s in
-// fp32. The warps' partial sums are added in a fixed order through shared memory.
+// Tensor-core path (2-, 3-, 4- and 8-bit codes, contiguous groups that are whole multiples of
+// 128 columns or one group per row, d_in a multiple of 128): work items are (row tile, 128-column
+// chunk); a warp's item is 8 mma.sync m16n8k16 (fp16 in, fp32 accumulate) per 16-row m-tile with
+// A = the codes and B = X (16 columns x 8 batch rows, lanes past the batch reading its last row).
+// Lane (g, t) holds rows g and g + 8 of each m-tile and the 32 columns [32 t, 32 t + 32) of the
+// chunk, exactly `bits` packed words per row. The codes enter A as fp16 subnormals decoded in
+// place (gemv_pairs.cuh: one AND per two codes), X takes the same column order with byte
+// permutes, and the scale and zero point are applied once per chunk in fp32:
+// Y += s 2^(24 - pos) sum_class - s z sum(x), the chunk's sum of x coming from MMAs with an
+// all-ones A. The grid is persistent and splits the items evenly over the SMs; partial sums of
+// a row tile are added into Y (zeroed first) with atomic adds.
 #include <cuda_fp16.h>
 
 #include "common.cuh"
@@ -182,7 +179,6 @@ dequant_gemv_kernel(const uint32_t* __restrict__ qweight, int n, int d, long lon
 // Tensor-core path
 // ---------------------------------------------------------------------------------------------
 constexpr int kChunk = 128;        // columns of one warp step (8 k-steps of 16)
-constexpr int kMmaMaxWarps = 8;
 
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                           uint32_t a3, uint32_t b0, uint32_t b1) {
