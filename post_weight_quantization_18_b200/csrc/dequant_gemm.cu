@@ -212,25 +212,33 @@ dequant_gemm_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
       int pb = 0;
       uint32_t par_phase = 0;
       bool ok = true;
+      // The row's fp16 (s, z) of the fold at column k0, read from global memory one fold before
+      // they are needed, so that the decoding never waits on them.
+      auto fold_params = [&](int row, int k0, uint16_t& sh, uint16_t& zh) {
+        sh = 0;
+        zh = 0;
+        if (row < args.N) {
+          const int gi = args.group_size > 0 ? k0 / args.group_size : 0;
+          const long long o = (long long)row * args.G + gi;
+          sh = __ldg(args.scales + o);
+          zh = __ldg(args.zeros + o);
+        }
+      };
       for (int t = blockIdx.x; t < args.n_tiles && ok && !*abort_flag; t += gridDim.x) {
         int tm, tn;
         tile_of(t, args, tm, tn);
         const int row = tn * BN + n;
+        uint16_t nxt_s, nxt_z;
+        fold_params(row, 0, nxt_s, nxt_z);
         for (int kb = 0; kb < nkb; ++kb) {
           if (kb % FOLD_KB == 0) {  // this fold's s * 2^24 and -s * z of the row
+            const float s = __half2float(__ushort_as_half(nxt_s));
+            // zero points are integers; another value is rounded to one
+            const float z = rintf(__half2float(__ushort_as_half(nxt_z)));
+            if (kb + FOLD_KB < nkb) fold_params(row, (kb + FOLD_KB) * BK, nxt_s, nxt_z);
             if (!gptq::mbar_wait(&par_empty[pb], par_phase ^ 1, abort_flag)) { ok = false; break; }
-            float sp = 0.f, nsz = 0.f;
-            if (row < args.N) {
-              const int gi = args.group_size > 0 ? (kb * BK) / args.group_size : 0;
-              const long long o = (long long)row * args.G + gi;
-              const float s = __half2float(__ushort_as_half(args.scales[o]));
-              // zero points are integers; another value is rounded to one
-              const float z = rintf(__half2float(__ushort_as_half(args.zeros[o])));
-              sp = s * 16777216.f;
-              nsz = -s * z;
-            }
-            par[pb * PAR_FLOATS + n] = sp;
-            par[pb * PAR_FLOATS + BN + n] = nsz;
+            par[pb * PAR_FLOATS + n] = s * 16777216.f;  // 0 past the rows: (s, z) = (0, 0)
+            par[pb * PAR_FLOATS + BN + n] = -s * z;
             __syncwarp();
             if (lane == 0) gptq::mbar_arrive(&par_full[pb]);
             if (++pb == 2) { pb = 0; par_phase ^= 1; }
