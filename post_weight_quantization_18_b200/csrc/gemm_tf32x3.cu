@@ -162,7 +162,7 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
           int kb0, kb1;
           tile_kb(tm, tn, args, nkb, kb0, kb1);
           for (int kb = kb0; kb < kb1; ++kb) {
-            if (!gptq::mbar_wait(&empty[stage], phase ^ 1, abort_flag)) break;
+            if (!gptq::mbar_wait_sleep(&empty[stage], phase ^ 1, abort_flag)) break;
             uint8_t* sa = smem + stage * STAGE_BYTES;
             uint8_t* sb = sa + TILE_BYTES;
             gptq::mbar_arrive_expect_tx(&full[stage], 2 * TILE_BYTES);
@@ -203,11 +203,14 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
           bool ok = true;
           for (int kc = kb0; kc < kb1 && ok; kc += KCB) {
             const int kc1 = min(kb1, kc + KCB);
-            if (!gptq::mbar_wait(&acc_empty[buf], acc_phase ^ 1, abort_flag)) { ok = false; break; }
+            if (!gptq::mbar_wait_sleep(&acc_empty[buf], acc_phase ^ 1, abort_flag)) {
+              ok = false;
+              break;
+            }
             gptq::tc_fence_after();
             const uint32_t d_tmem = tmem_base + ACC_COL + (uint32_t)(buf * BN);
             for (int kb = kc; kb < kc1; ++kb) {
-              if (!gptq::mbar_wait(&conv[stage], phase, abort_flag)) { ok = false; break; }
+              if (!gptq::mbar_wait_sleep(&conv[stage], phase, abort_flag)) { ok = false; break; }
               gptq::tc_fence_after();
               const uint32_t b_hi = gptq::smem_u32(smem + stage * STAGE_BYTES + TILE_BYTES);
               const uint32_t b_lo = b_hi + TILE_BYTES;
@@ -250,7 +253,7 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
         int kb0, kb1;
         tile_kb(tm, tn, args, nkb, kb0, kb1);
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!gptq::mbar_wait(&full[stage], phase, abort_flag)) break;
+          if (!gptq::mbar_wait_sleep(&full[stage], phase, abort_flag)) break;
           const uint8_t* sa = smem + stage * STAGE_BYTES;
           uint32_t hi[32], lo[32];
           if (args.a_mn) {
@@ -315,7 +318,7 @@ gemm_tf32x3_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constan
         for (int e = 0; e < EPI_COLS; ++e) acc[e] = 0.f;  // 0 + x is x exactly: no select
         bool ok = true;
         for (int kc = kb0; kc < kb1; kc += KCB) {
-          if (!gptq::mbar_wait(&acc_full[buf], acc_phase, abort_flag)) { ok = false; break; }
+          if (!gptq::mbar_wait_sleep(&acc_full[buf], acc_phase, abort_flag)) { ok = false; break; }
           gptq::tc_fence_after();
 #pragma unroll
           for (int q = 0; q < EPI_COLS / 32; ++q) {
