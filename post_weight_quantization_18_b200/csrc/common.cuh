@@ -75,8 +75,9 @@ GPTQ_DEV bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t suspe
   return ok != 0;
 }
 // Suspend hint of the waits in the 3xTF32 GEMM: its waiting warps then poll far less often.
-// Measured on B200 at the 1 kW cap: the 8192^3 GEMM 177 -> 185 TFLOP/s; the SYRK lost 9 % with
-// it and the dequantizing GEMM 2.5 %, so those kernels poll without it.
+// Measured on B200 at the 1 kW cap, 8192^3: 177 -> 185 TFLOP/s on one box, no change beyond
+// 1 % on another; the SYRK lost 9 % with it and the dequantizing GEMM 2.5 %, so those kernels
+// poll without it.
 constexpr uint32_t kSleepNs = 1000;
 
 // Wait for the phase with the given parity to complete. Returns false (and raises *abort) if
